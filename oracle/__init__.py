@@ -1,0 +1,214 @@
+"""CPU oracle for C = relu(A . op(B)) -- TEST INFRASTRUCTURE ONLY.
+
+Only the test suite, ``__graft_entry__.smoke()`` and the benchmark's CPU
+baseline leg may import this package.  The CUDA library never loads it, and
+it shares no code with the CUDA path: the arithmetic lives in ``oracle.c``
+(plain C, fp64, sequential-k sums), built here with gcc.
+
+What it follows (the matmul_relu definition on the TileLang technical notes
+page, sections 3.2 and 3.3, and the tiled GEMM example of the "From TVM to
+TileLang" essay, section 2):
+
+    ref[i, j] = relu( sum_k double(A[i, k]) * double(op(B)[k, j]) )
+
+with op(B) = B for B stored (K, N) and op(B) = B^T for B stored (N, K)
+(``trans_b``).  The result is returned unrounded as float64.  ``round_output``
+gives the oracle's own image in the output dtype, for reporting only; parity
+is judged against the unrounded value.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+F16 = 0
+BF16 = 1
+
+_CFLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-fopenmp", "-fPIC", "-shared",
+           "-Wall", "-Wextra"]
+
+
+def build(force: bool = False, src: str = _SRC, lib: str = _LIB) -> str:
+    """Compile ``src`` (default oracle.c) into ``lib`` if stale; return the path."""
+    if force or not os.path.exists(lib) or os.path.getmtime(lib) < os.path.getmtime(src):
+        tmp = lib + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *_CFLAGS, "-o", tmp, src, "-lm"])
+        os.replace(tmp, lib)
+    return lib
+
+
+def _bind(path: str):
+    lib = ctypes.CDLL(path)
+    i64, i32, vp = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p
+    lib.oracle_decode.argtypes = [vp, vp, i64, i32]
+    lib.oracle_gemm_relu.argtypes = [vp, vp, vp, i64, i64, i64, i32, i32, i32, i32]
+    lib.oracle_gemm_relu_sampled.argtypes = [vp, vp, vp, vp, i64, vp, i64, i64, i64,
+                                             i32, i32, i32, i32]
+    lib.oracle_gemm_relu_rows.argtypes = [vp, vp, vp, i64, vp, i64, i64, i64,
+                                          i32, i32, i32, i32]
+    for f in (lib.oracle_decode, lib.oracle_gemm_relu, lib.oracle_gemm_relu_sampled,
+              lib.oracle_gemm_relu_rows):
+        f.restype = i32
+    lib.oracle_num_threads.restype = i32
+    lib.oracle_num_threads.argtypes = []
+    return lib
+
+
+def _code(dtype: torch.dtype) -> int:
+    if dtype == torch.float16:
+        return F16
+    if dtype == torch.bfloat16:
+        return BF16
+    raise TypeError(f"oracle inputs must be float16 or bfloat16, got {dtype}")
+
+
+def _bits(t: torch.Tensor) -> np.ndarray:
+    """The raw 16-bit patterns of a CPU fp16/bf16 tensor, contiguous."""
+    if t.device.type != "cpu":
+        raise ValueError("oracle inputs must be CPU tensors")
+    return np.ascontiguousarray(t.contiguous().view(torch.int16).numpy()).view(np.uint16)
+
+
+def _shape(A: torch.Tensor, B: torch.Tensor, trans_b: bool):
+    if A.dim() != 2 or B.dim() != 2:
+        raise ValueError("A and B must be 2-D")
+    if A.dtype != B.dtype:
+        raise TypeError("A and B must have the same dtype")
+    M, K = A.shape
+    if trans_b:
+        N, Kb = B.shape
+    else:
+        Kb, N = B.shape
+    if Kb != K:
+        raise ValueError(f"inner dimensions differ: A has K={K}, B has K={Kb}")
+    return int(M), int(N), int(K)
+
+
+class Oracle:
+    """The oracle entry points bound to one compiled copy of oracle.c."""
+
+    def __init__(self, path: str):
+        self.path = path
+        self.lib = _bind(path)
+
+    def num_threads(self) -> int:
+        """Threads the OpenMP loops use by default on this host."""
+        return int(self.lib.oracle_num_threads())
+
+    def decode(self, bits: np.ndarray, dtype: torch.dtype) -> np.ndarray:
+        """Widen raw fp16/bf16 bit patterns (uint16) to float64 with the oracle's decoder."""
+        src = np.ascontiguousarray(bits, dtype=np.uint16)
+        out = np.empty(src.shape, dtype=np.float64)
+        rc = self.lib.oracle_decode(src.ctypes.data, out.ctypes.data, src.size, _code(dtype))
+        if rc != 0:
+            raise RuntimeError(f"oracle_decode failed ({rc})")
+        return out
+
+    def gemm_relu(self, A: torch.Tensor, B: torch.Tensor, trans_b: bool = False,
+                  relu: bool = True, threads: int = 0) -> np.ndarray:
+        """Full reference product as float64 (M, N)."""
+        M, N, K = _shape(A, B, trans_b)
+        a, b = _bits(A), _bits(B)
+        out = np.zeros((M, N), dtype=np.float64)
+        rc = self.lib.oracle_gemm_relu(a.ctypes.data, b.ctypes.data, out.ctypes.data, M, N, K,
+                                       _code(A.dtype), int(bool(trans_b)), int(bool(relu)),
+                                       int(threads))
+        if rc != 0:
+            raise RuntimeError(f"oracle_gemm_relu failed ({rc})")
+        return out
+
+    def gemm_relu_sampled(self, A: torch.Tensor, B: torch.Tensor, rows, cols,
+                          trans_b: bool = False, relu: bool = True,
+                          threads: int = 0) -> np.ndarray:
+        """Reference values at the listed (rows[t], cols[t]) positions, float64."""
+        M, N, K = _shape(A, B, trans_b)
+        r = np.ascontiguousarray(rows, dtype=np.int64)
+        c = np.ascontiguousarray(cols, dtype=np.int64)
+        if r.shape != c.shape:
+            raise ValueError("rows and cols must have the same length")
+        a, b = _bits(A), _bits(B)
+        out = np.zeros(r.shape, dtype=np.float64)
+        rc = self.lib.oracle_gemm_relu_sampled(a.ctypes.data, b.ctypes.data, r.ctypes.data,
+                                               c.ctypes.data, r.size, out.ctypes.data, M, N,
+                                               K, _code(A.dtype), int(bool(trans_b)),
+                                               int(bool(relu)), int(threads))
+        if rc != 0:
+            raise RuntimeError(f"oracle_gemm_relu_sampled failed ({rc})")
+        return out
+
+    def gemm_relu_rows(self, A: torch.Tensor, B: torch.Tensor, rows, trans_b: bool = False,
+                       relu: bool = True, threads: int = 0) -> np.ndarray:
+        """Whole reference rows, float64 (len(rows), N)."""
+        M, N, K = _shape(A, B, trans_b)
+        r = np.ascontiguousarray(rows, dtype=np.int64)
+        a, b = _bits(A), _bits(B)
+        out = np.zeros((r.size, N), dtype=np.float64)
+        rc = self.lib.oracle_gemm_relu_rows(a.ctypes.data, b.ctypes.data, r.ctypes.data,
+                                            r.size, out.ctypes.data, M, N, K, _code(A.dtype),
+                                            int(bool(trans_b)), int(bool(relu)), int(threads))
+        if rc != 0:
+            raise RuntimeError(f"oracle_gemm_relu_rows failed ({rc})")
+        return out
+
+    def gemm_relu_cols(self, A: torch.Tensor, B: torch.Tensor, cols, trans_b: bool = False,
+                       relu: bool = True, threads: int = 0) -> np.ndarray:
+        """Whole reference columns, float64 (M, len(cols)), via the sampled routine."""
+        M, N, _ = _shape(A, B, trans_b)
+        c = np.asarray(cols, dtype=np.int64)
+        rr = np.repeat(np.arange(M, dtype=np.int64)[:, None], c.size, axis=1).ravel()
+        cc = np.repeat(c[None, :], M, axis=0).ravel()
+        return self.gemm_relu_sampled(A, B, rr, cc, trans_b, relu, threads).reshape(M, c.size)
+
+
+def _default() -> Oracle:
+    global _lib
+    with _lock:
+        if _lib is None:
+            _lib = Oracle(build())
+    return _lib
+
+
+def num_threads() -> int:
+    return _default().num_threads()
+
+
+def decode(bits, dtype):
+    return _default().decode(bits, dtype)
+
+
+def gemm_relu(A, B, trans_b=False, relu=True, threads=0):
+    return _default().gemm_relu(A, B, trans_b, relu, threads)
+
+
+def gemm_relu_sampled(A, B, rows, cols, trans_b=False, relu=True, threads=0):
+    return _default().gemm_relu_sampled(A, B, rows, cols, trans_b, relu, threads)
+
+
+def gemm_relu_rows(A, B, rows, trans_b=False, relu=True, threads=0):
+    return _default().gemm_relu_rows(A, B, rows, trans_b, relu, threads)
+
+
+def gemm_relu_cols(A, B, cols, trans_b=False, relu=True, threads=0):
+    return _default().gemm_relu_cols(A, B, cols, trans_b, relu, threads)
+
+
+def round_output(ref: np.ndarray, out_dtype: torch.dtype) -> torch.Tensor:
+    """The oracle's image in the output dtype (reporting only; parity uses ``ref``).
+
+    float64 -> float16 goes through numpy's direct round-to-nearest-even
+    conversion; float64 -> bfloat16 and float32 go through torch's casts.
+    """
+    if out_dtype == torch.float16:
+        return torch.from_numpy(np.asarray(ref, dtype=np.float64).astype(np.float16))
+    return torch.from_numpy(np.asarray(ref, dtype=np.float64)).to(out_dtype)

@@ -1,0 +1,274 @@
+/*
+ * oracle.c -- CPU oracle for the fused GEMM + ReLU hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
+ * call this file; only the test suite, the smoke check and the benchmark's
+ * CPU-baseline leg use it.  It shares no code, header, table or helper with
+ * the CUDA library.
+ *
+ * What it computes (the plain definition, written out):
+ *
+ *     ref[i][j] = relu( sum_{k=0}^{K-1} a(i,k) * b(k,j) )
+ *
+ * where a(i,k) = A[i*K + k] (A is M x K, row-major) and
+ *     b(k,j) = B[k*N + j]  when trans_b == 0  (B stored K x N, row-major),
+ *     b(k,j) = B[j*K + k]  when trans_b == 1  (B stored N x K, row-major),
+ * relu(x) = x > 0 ? x : 0, or the identity when relu == 0.
+ *
+ * Source of the definition:
+ *   - TileLang technical notes page, section 3.2 "GPU minimal example":
+ *     the matmul_relu kernel clears a fp32 accumulator, accumulates A*B tile
+ *     by tile over the whole K loop, applies max(C, 0) element-wise, then
+ *     copies the result out (fp16 in, fp32 accumulate, fp16 out).
+ *   - same page, section 3.3 "the same GEMM on Ascend 950": B is given as
+ *     (N, K) and the product is taken with transpose_B = True; bf16 in,
+ *     fp32 out, ReLU before the store.
+ *   - "From TVM to TileLang" essay, section 2: the tiled GEMM example without
+ *     the ReLU (relu == 0 here).
+ *
+ * Arithmetic: each 16-bit input is widened EXACTLY to double (every binary16
+ * and bfloat16 value is representable in binary64), every product of two
+ * such values is exact in binary64 (11+11 or 8+8 significand bits), and the
+ * K products of one output are summed in increasing k order in binary64.
+ * No blocking, no reordering, no fused multiply-add (build with
+ * -ffp-contract=off).  The result is returned as double, unrounded; the
+ * output cast to fp16/bf16/fp32 is not applied here.
+ *
+ * The loop order i-k-j used for trans_b == 0 is only a memory-order choice:
+ * every output still receives its K terms one at a time in increasing k, so
+ * the result is bit-identical to the textbook i-j-k triple loop.
+ */
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <math.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+enum { ORACLE_F16 = 0, ORACLE_BF16 = 1 };
+
+/* IEEE-754 binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction
+ * bits.  Exponent 0 encodes zero/subnormals (value = frac * 2^-24), exponent
+ * 31 encodes infinity (frac == 0) or NaN. */
+static double decode_f16(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int expo = (h >> 10) & 0x1f;
+    int frac = h & 0x3ff;
+    double v;
+    if (expo == 0)
+        v = ldexp((double)frac, -24);
+    else if (expo == 31)
+        v = frac ? NAN : INFINITY;
+    else
+        v = ldexp((double)(frac | 0x400), expo - 25);
+    return sign ? -v : v;
+}
+
+/* bfloat16: the upper 16 bits of an IEEE-754 binary32 (1 sign bit, 8
+ * exponent bits with bias 127, 7 fraction bits). */
+static double decode_bf16(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int expo = (h >> 7) & 0xff;
+    int frac = h & 0x7f;
+    double v;
+    if (expo == 0)
+        v = ldexp((double)frac, -133);
+    else if (expo == 255)
+        v = frac ? NAN : INFINITY;
+    else
+        v = ldexp((double)(frac | 0x80), expo - 134);
+    return sign ? -v : v;
+}
+
+static int decode_array(const uint16_t *src, double *dst, int64_t n, int dtype)
+{
+    if (dtype == ORACLE_F16) {
+        for (int64_t i = 0; i < n; ++i) dst[i] = decode_f16(src[i]);
+    } else if (dtype == ORACLE_BF16) {
+        for (int64_t i = 0; i < n; ++i) dst[i] = decode_bf16(src[i]);
+    } else {
+        return -1;
+    }
+    return 0;
+}
+
+static double apply_relu(double x, int relu)
+{
+    if (!relu) return x;
+    return x > 0.0 ? x : 0.0;
+}
+
+/* Decode n 16-bit values of the given type to double (exposed so the tests
+ * can pin the decoder against every bit pattern). */
+int oracle_decode(const uint16_t *src, double *dst, int64_t n, int dtype)
+{
+    if (n < 0 || (n > 0 && (!src || !dst))) return -1;
+    return decode_array(src, dst, n, dtype);
+}
+
+static void set_threads(int nthreads)
+{
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* Per-thread scratch for the row loops: nt slices of (K + N) doubles. */
+static double *alloc_scratch(int64_t K, int64_t N, int *nt_out)
+{
+    int nt = oracle_num_threads();
+    if (nt < 1) nt = 1;
+    *nt_out = nt;
+    size_t per = (size_t)(K + N + 1);
+    return (double *)malloc(sizeof(double) * per * (size_t)nt);
+}
+
+static int thread_id(void)
+{
+#ifdef _OPENMP
+    return omp_get_thread_num();
+#else
+    return 0;
+#endif
+}
+
+/* One output row: dst[j] = relu(sum_k arow[k] * b(k,j)) for j in [j0, j1),
+ * each sum taken in increasing k.  For trans_b == 0 the K x N matrix Bd is
+ * walked row by row with dst as the running sums (memory order only). */
+static void row_product(const double *arow, const double *Bd, double *dst,
+                        int64_t N, int64_t K, int64_t j0, int64_t j1,
+                        int trans_b, int relu)
+{
+    if (!trans_b) {
+        for (int64_t j = j0; j < j1; ++j) dst[j] = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            const double a = arow[k];
+            const double *brow = Bd + k * N;
+            for (int64_t j = j0; j < j1; ++j) dst[j] = dst[j] + a * brow[j];
+        }
+        for (int64_t j = j0; j < j1; ++j) dst[j] = apply_relu(dst[j], relu);
+    } else {
+        for (int64_t j = j0; j < j1; ++j) {
+            const double *bcol = Bd + j * K; /* row j of the stored (N, K) B */
+            double s = 0.0;
+            for (int64_t k = 0; k < K; ++k) s = s + arow[k] * bcol[k];
+            dst[j] = apply_relu(s, relu);
+        }
+    }
+}
+
+/* Full product: C (M x N, double, row-major) = relu(A * op(B)).
+ * Returns 0 on success, -1 on bad arguments, -2 on allocation failure. */
+int oracle_gemm_relu(const uint16_t *A, const uint16_t *B, double *C,
+                     int64_t M, int64_t N, int64_t K,
+                     int in_dtype, int trans_b, int relu, int nthreads)
+{
+    if (M < 0 || N < 0 || K < 0) return -1;
+    if (in_dtype != ORACLE_F16 && in_dtype != ORACLE_BF16) return -1;
+    if (M == 0 || N == 0) return 0;
+    if (!C || (K > 0 && (!A || !B))) return -1;
+    set_threads(nthreads);
+
+    double *Bd = (double *)malloc(sizeof(double) * (size_t)(K > 0 ? K * N : 1));
+    int nt = 1;
+    double *scratch = alloc_scratch(K, N, &nt);
+    if (!Bd || !scratch) { free(Bd); free(scratch); return -2; }
+    decode_array(B, Bd, K * N, in_dtype);   /* exact widening, once */
+
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = 0; i < M; ++i) {
+        double *arow = scratch + (size_t)thread_id() * (size_t)(K + N + 1);
+        decode_array(A + i * K, arow, K, in_dtype);
+        row_product(arow, Bd, C + i * N, N, K, 0, N, trans_b, relu);
+    }
+    free(scratch);
+    free(Bd);
+    return 0;
+}
+
+/* Selected outputs only: out[t] = ref[rows[t]][cols[t]] for t < count, each
+ * one the same sequential-k sum as above.  Used where the full product would
+ * take the CPU too long. */
+int oracle_gemm_relu_sampled(const uint16_t *A, const uint16_t *B,
+                             const int64_t *rows, const int64_t *cols,
+                             int64_t count, double *out,
+                             int64_t M, int64_t N, int64_t K,
+                             int in_dtype, int trans_b, int relu, int nthreads)
+{
+    if (M < 0 || N < 0 || K < 0 || count < 0) return -1;
+    if (in_dtype != ORACLE_F16 && in_dtype != ORACLE_BF16) return -1;
+    if (count == 0) return 0;
+    if (!rows || !cols || !out || (K > 0 && (!A || !B))) return -1;
+    for (int64_t t = 0; t < count; ++t)
+        if (rows[t] < 0 || rows[t] >= M || cols[t] < 0 || cols[t] >= N) return -1;
+    set_threads(nthreads);
+
+    #pragma omp parallel for schedule(dynamic, 16)
+    for (int64_t t = 0; t < count; ++t) {
+        const int64_t i = rows[t], j = cols[t];
+        double s = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            uint16_t av = A[i * K + k];
+            uint16_t bv = trans_b ? B[j * K + k] : B[k * N + j];
+            double a = in_dtype == ORACLE_F16 ? decode_f16(av) : decode_bf16(av);
+            double b = in_dtype == ORACLE_F16 ? decode_f16(bv) : decode_bf16(bv);
+            s = s + a * b;
+        }
+        out[t] = apply_relu(s, relu);
+    }
+    return 0;
+}
+
+/* Whole rows: out (nrows x N) = ref[rows[r]][:].  Same arithmetic as the
+ * full product, restricted to the listed rows; the N outputs of one row are
+ * split over the threads in contiguous ranges. */
+int oracle_gemm_relu_rows(const uint16_t *A, const uint16_t *B,
+                          const int64_t *rows, int64_t nrows, double *out,
+                          int64_t M, int64_t N, int64_t K,
+                          int in_dtype, int trans_b, int relu, int nthreads)
+{
+    if (M < 0 || N < 0 || K < 0 || nrows < 0) return -1;
+    if (in_dtype != ORACLE_F16 && in_dtype != ORACLE_BF16) return -1;
+    if (nrows == 0 || N == 0) return 0;
+    if (!rows || !out || (K > 0 && (!A || !B))) return -1;
+    for (int64_t r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= M) return -1;
+    set_threads(nthreads);
+
+    double *Bd = (double *)malloc(sizeof(double) * (size_t)(K > 0 ? K * N : 1));
+    double *arow = (double *)malloc(sizeof(double) * (size_t)(K > 0 ? K : 1));
+    if (!Bd || !arow) { free(Bd); free(arow); return -2; }
+    decode_array(B, Bd, K * N, in_dtype);
+
+    for (int64_t r = 0; r < nrows; ++r) {
+        decode_array(A + rows[r] * K, arow, K, in_dtype);
+        double *dst = out + r * N;
+        #pragma omp parallel
+        {
+#ifdef _OPENMP
+            const int64_t nt = omp_get_num_threads(), t = omp_get_thread_num();
+#else
+            const int64_t nt = 1, t = 0;
+#endif
+            const int64_t j0 = N * t / nt, j1 = N * (t + 1) / nt;
+            row_product(arow, Bd, dst, N, K, j0, j1, trans_b, relu);
+        }
+    }
+    free(arow);
+    free(Bd);
+    return 0;
+}

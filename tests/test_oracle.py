@@ -1,0 +1,342 @@
+"""Pins for the CPU oracle (no GPU).
+
+Each test checks the oracle against something other than itself: a library
+routine on the decoder, closed forms of the matmul_relu definition (TileLang
+notes, sections 3.2 / 3.3), exact rational arithmetic on tiny shapes, exact
+integer arithmetic, a hand-worked example, and a textbook fp64 product.  The
+mutation test at the end plants plausible mistakes in a copy of the oracle
+and checks that some pin catches each one.
+"""
+from __future__ import annotations
+
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+from tests.parity_util import read_golden
+from tiled_tensor_core_04_b200 import workloads as wl
+
+DTYPES = [torch.float16, torch.bfloat16]
+
+
+# --------------------------------------------------------------------------
+# the 16-bit decoder, against every bit pattern
+# --------------------------------------------------------------------------
+
+def test_decode_f16_every_pattern(oracle_mod):
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    got = oracle_mod.decode(bits, torch.float16)
+    want = bits.view(np.float16).astype(np.float64)
+    nan = np.isnan(want)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], want[~nan])
+    # signed zeros decode with their sign
+    assert np.signbit(got[0x8000]) and not np.signbit(got[0])
+
+
+def test_decode_bf16_every_pattern(oracle_mod):
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    got = oracle_mod.decode(bits, torch.bfloat16)
+    want = torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).double().numpy()
+    nan = np.isnan(want)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], want[~nan])
+
+
+# --------------------------------------------------------------------------
+# closed forms of the definition
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("trans_b", [False, True])
+@pytest.mark.parametrize("M,N,K", [(1, 1, 1), (3, 5, 7), (17, 9, 2050), (8, 33, 256)])
+def test_ones_give_K(oracle_mod, dtype, trans_b, M, N, K):
+    A = torch.ones(M, K, dtype=dtype)
+    B = torch.ones((N, K) if trans_b else (K, N), dtype=dtype)
+    ref = oracle_mod.gemm_relu(A, B, trans_b=trans_b, relu=True)
+    assert np.all(ref == float(K))
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("trans_b", [False, True])
+@pytest.mark.parametrize("relu", [False, True])
+def test_identity_B_gives_relu_A(oracle_mod, dtype, trans_b, relu):
+    M, K = 37, 48
+    A, _ = wl.make_inputs(M, K, K, dtype, False, "uniform", seed=11)
+    B = torch.eye(K, dtype=dtype)                      # I == I^T
+    ref = oracle_mod.gemm_relu(A, B, trans_b=trans_b, relu=relu)
+    a = A.double().numpy()
+    want = np.where(a > 0, a, 0.0) if relu else a
+    assert np.array_equal(ref, want)
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+def test_permutation_B_permutes_columns(oracle_mod, dtype):
+    # b(k, j) = 1 iff k == perm[j]  ->  ref[:, j] = relu(A[:, perm[j]])
+    M, K = 19, 40
+    perm = np.random.default_rng(5).permutation(K)
+    A, _ = wl.make_inputs(M, K, K, dtype, False, "uniform", seed=12)
+    B = torch.zeros(K, K, dtype=dtype)
+    B[torch.from_numpy(perm), torch.arange(K)] = 1
+    ref = oracle_mod.gemm_relu(A, B, trans_b=False, relu=True)
+    a = A.double().numpy()[:, perm]
+    assert np.array_equal(ref, np.maximum(a, 0.0))
+    ref_t = oracle_mod.gemm_relu(A, B.t().contiguous(), trans_b=True, relu=True)
+    assert np.array_equal(ref_t, ref)
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("trans_b", [False, True])
+def test_all_negative_product_gives_zero(oracle_mod, dtype, trans_b):
+    M, N, K = 21, 34, 55
+    A, B = wl.make_inputs(M, N, K, dtype, trans_b, "uniform", seed=13)
+    A, B = A.abs(), -B.abs()
+    ref = oracle_mod.gemm_relu(A, B, trans_b=trans_b, relu=True)
+    assert np.all(ref == 0.0)
+    plain = oracle_mod.gemm_relu(A, B, trans_b=trans_b, relu=False)
+    assert np.all(plain <= 0.0) and np.any(plain < 0.0)
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+def test_zero_K_gives_zero(oracle_mod, dtype):
+    A = torch.zeros(4, 0, dtype=dtype)
+    B = torch.zeros(0, 6, dtype=dtype)
+    assert np.all(oracle_mod.gemm_relu(A, B) == 0.0)
+
+
+# --------------------------------------------------------------------------
+# invariants
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("trans_b", [False, True])
+def test_invariants(oracle_mod, dtype, trans_b):
+    M, N, K = 29, 31, 67
+    A, B = wl.make_inputs(M, N, K, dtype, trans_b, "uniform", seed=14)
+    plain = oracle_mod.gemm_relu(A, B, trans_b=trans_b, relu=False)
+    rel = oracle_mod.gemm_relu(A, B, trans_b=trans_b, relu=True)
+    assert np.all(rel >= 0.0)
+    assert np.array_equal(rel, np.maximum(plain, 0.0))      # relu after the full sum
+    neg = oracle_mod.gemm_relu(-A, B, trans_b=trans_b, relu=False)
+    assert np.array_equal(neg, -plain)                         # negation is exact
+    negb = oracle_mod.gemm_relu(A, -B, trans_b=trans_b, relu=False)
+    assert np.array_equal(negb, -plain)
+    # scaling by a power of two is exact
+    twice = oracle_mod.gemm_relu(A * 2, B, trans_b=trans_b, relu=True)
+    assert np.array_equal(twice, 2 * rel)
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+def test_trans_b_is_the_transpose(oracle_mod, dtype):
+    M, N, K = 23, 45, 70
+    A, B = wl.make_inputs(M, N, K, dtype, False, "uniform", seed=15)
+    r0 = oracle_mod.gemm_relu(A, B, trans_b=False)
+    r1 = oracle_mod.gemm_relu(A, B.t().contiguous(), trans_b=True)
+    assert np.array_equal(r0, r1)
+
+
+def test_row_and_column_linearity(oracle_mod):
+    # ref_plain[i, :] depends only on A[i, :]: swapping rows of A swaps rows.
+    A, B = wl.make_inputs(12, 10, 33, torch.float16, False, "uniform", seed=16)
+    plain = oracle_mod.gemm_relu(A, B, relu=False)
+    p = np.random.default_rng(1).permutation(12)
+    plain_p = oracle_mod.gemm_relu(A[torch.from_numpy(p)].contiguous(), B, relu=False)
+    assert np.array_equal(plain_p, plain[p])
+    q = np.random.default_rng(2).permutation(10)
+    plain_q = oracle_mod.gemm_relu(A, B[:, torch.from_numpy(q)].contiguous(), relu=False)
+    assert np.array_equal(plain_q, plain[:, q])
+
+
+# --------------------------------------------------------------------------
+# exact arithmetic
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("trans_b", [False, True])
+@pytest.mark.parametrize("M,N,K", [(1, 1, 1), (2, 3, 5), (7, 13, 17), (17, 1, 16),
+                                   (65, 130, 257)])
+def test_small_integers_are_exact(oracle_mod, dtype, trans_b, M, N, K):
+    A, B = wl.small_int_inputs(M, N, K, dtype, trans_b, seed=M * 100 + N)
+    a = A.to(torch.int64).numpy()
+    b = B.to(torch.int64).numpy()
+    exact = a @ (b.T if trans_b else b)                      # integer arithmetic
+    for relu in (False, True):
+        ref = oracle_mod.gemm_relu(A, B, trans_b=trans_b, relu=relu)
+        want = np.maximum(exact, 0) if relu else exact
+        assert np.array_equal(ref, want.astype(np.float64))
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("trans_b", [False, True])
+@pytest.mark.parametrize("M,N,K", [(1, 1, 1), (3, 2, 5), (5, 7, 11), (4, 3, 17),
+                                   (17, 13, 2)])
+def test_brute_force_rationals(oracle_mod, dtype, trans_b, M, N, K):
+    """Exact sum in Fraction; the fp64 sequential sum is within (K-1) 2^-53 sum|ab|."""
+    A, B = wl.make_inputs(M, N, K, dtype, trans_b, "uniform", seed=K * 7 + M)
+    av = [[Fraction(float(v)) for v in row] for row in A.double().tolist()]
+    bv = [[Fraction(float(v)) for v in row] for row in B.double().tolist()]
+    ref = oracle_mod.gemm_relu(A, B, trans_b=trans_b, relu=False)
+    rel = oracle_mod.gemm_relu(A, B, trans_b=trans_b, relu=True)
+    for i in range(M):
+        for j in range(N):
+            terms = [av[i][k] * (bv[j][k] if trans_b else bv[k][j]) for k in range(K)]
+            exact = sum(terms, Fraction(0))
+            bound = (K - 1) * 2.0 ** -53 * float(sum(abs(t) for t in terms))
+            assert abs(Fraction(ref[i, j]) - exact) <= Fraction(bound)
+            assert rel[i, j] == (ref[i, j] if ref[i, j] > 0 else 0.0)
+
+
+def test_golden_worked_example(oracle_mod):
+    g = read_golden("worked_example.txt")
+    for dtype in DTYPES:
+        A = torch.from_numpy(g["A"]).to(dtype)
+        Bkn = torch.from_numpy(g["B_KN"]).to(dtype)
+        Bnk = torch.from_numpy(g["B_NK"]).to(dtype)
+        assert np.array_equal(oracle_mod.gemm_relu(A, Bkn, relu=False), g["C_plain"])
+        assert np.array_equal(oracle_mod.gemm_relu(A, Bkn, relu=True), g["C_relu"])
+        assert np.array_equal(oracle_mod.gemm_relu(A, Bnk, trans_b=True, relu=True), g["C_relu"])
+
+
+@pytest.mark.parametrize("trans_b", [False, True])
+@pytest.mark.parametrize("M,N,K", [(64, 96, 128), (130, 257, 300), (512, 256, 512)])
+def test_textbook_fp64_product(oracle_mod, trans_b, M, N, K):
+    A, B = wl.make_inputs(M, N, K, torch.float16, trans_b, "uniform", seed=M + N + K)
+    Bop = B.double().t() if trans_b else B.double()
+    want = (A.double() @ Bop).clamp_min(0).numpy()
+    scale = (A.double().abs() @ Bop.abs()).numpy()
+    ref = oracle_mod.gemm_relu(A, B, trans_b=trans_b)
+    assert np.all(np.abs(ref - want) <= 1e-12 * scale + 1e-300)
+
+
+# --------------------------------------------------------------------------
+# the sampled / row / column entry points agree with the full product
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("trans_b", [False, True])
+def test_partial_entry_points_match_full(oracle_mod, dtype, trans_b):
+    M, N, K = 70, 90, 130
+    A, B = wl.make_inputs(M, N, K, dtype, trans_b, "normal", seed=17)
+    full = oracle_mod.gemm_relu(A, B, trans_b=trans_b)
+    r, c = wl.sample_positions(M, N, seed=3, count=500)
+    assert np.array_equal(oracle_mod.gemm_relu_sampled(A, B, r, c, trans_b=trans_b), full[r, c])
+    rows = [0, 1, 63, 64, 69]
+    assert np.array_equal(oracle_mod.gemm_relu_rows(A, B, rows, trans_b=trans_b), full[rows])
+    cols = [0, 5, 64, 89]
+    assert np.array_equal(oracle_mod.gemm_relu_cols(A, B, cols, trans_b=trans_b), full[:, cols])
+    for th in (1, 3):
+        assert np.array_equal(oracle_mod.gemm_relu(A, B, trans_b=trans_b, threads=th), full)
+
+
+def test_bad_arguments(oracle_mod):
+    A = torch.zeros(3, 4, dtype=torch.float16)
+    with pytest.raises(ValueError):
+        oracle_mod.gemm_relu(A, torch.zeros(5, 6, dtype=torch.float16))
+    with pytest.raises(TypeError):
+        oracle_mod.gemm_relu(A, torch.zeros(4, 6, dtype=torch.bfloat16))
+    with pytest.raises(TypeError):
+        oracle_mod.gemm_relu(A.float(), torch.zeros(4, 6))
+    with pytest.raises(RuntimeError):
+        oracle_mod.gemm_relu_sampled(A, torch.zeros(4, 6, dtype=torch.float16), [3], [0])
+
+
+# --------------------------------------------------------------------------
+# the seeded input recipe
+# --------------------------------------------------------------------------
+
+def test_inputs_are_seeded_and_shaped():
+    A1, B1 = wl.make_inputs(33, 17, 65, torch.float16, False, "uniform", seed=9)
+    A2, B2 = wl.make_inputs(33, 17, 65, torch.float16, False, "uniform", seed=9)
+    A3, _ = wl.make_inputs(33, 17, 65, torch.float16, False, "uniform", seed=10)
+    assert torch.equal(A1, A2) and torch.equal(B1, B2) and not torch.equal(A1, A3)
+    assert A1.shape == (33, 65) and B1.shape == (65, 17)
+    assert float(A1.abs().max()) <= 1.0
+    _, Bt = wl.make_inputs(8, 300, 400, torch.bfloat16, True, "normal", seed=3)
+    assert Bt.shape == (300, 400) and Bt.dtype == torch.bfloat16
+    assert 0.09 < float(Bt.float().std()) < 0.11
+
+
+def test_workload_table():
+    w = wl.WORKLOADS[wl.HEADLINE]
+    assert (w.M, w.N, w.K) == (8192, 8192, 8192) and w.in_dtype == torch.float16
+    assert w.flops == 2 * 8192 ** 3
+    bt = wl.WORKLOADS["bt8192x7168x8192_bf16_f32"]
+    assert bt.trans_b and bt.out_dtype == torch.float32 and bt.in_dtype == torch.bfloat16
+    assert bt.N == 32 * 224 and bt.M == 32 * 256
+    assert [w.seed for w in wl.WORKLOADS.values()] == [0, 1, 2, 3, 4, 4, 4]
+
+
+# --------------------------------------------------------------------------
+# planted mistakes: each mutant copy of oracle.c must fail some pin
+# --------------------------------------------------------------------------
+
+def _pins_pass(o) -> bool:
+    """A compact run of the pins above against one compiled oracle; True if all hold."""
+    try:
+        bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+        f16 = bits.view(np.float16).astype(np.float64)
+        got = o.decode(bits, torch.float16)
+        ok = np.isnan(f16)
+        if not (np.array_equal(np.isnan(got), ok) and np.array_equal(got[~ok], f16[~ok])):
+            return False
+        bf = torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).double().numpy()
+        got = o.decode(bits, torch.bfloat16)
+        ok = np.isnan(bf)
+        if not (np.array_equal(np.isnan(got), ok) and np.array_equal(got[~ok], bf[~ok])):
+            return False
+        for dtype in DTYPES:
+            for tb in (False, True):
+                M, N, K = 9, 11, 37
+                A = torch.ones(M, K, dtype=dtype)
+                B = torch.ones((N, K) if tb else (K, N), dtype=dtype)
+                if not np.all(o.gemm_relu(A, B, tb) == K):
+                    return False
+                A, B = wl.small_int_inputs(7, 13, 17, dtype, tb, seed=3)
+                a, b = A.to(torch.int64).numpy(), B.to(torch.int64).numpy()
+                exact = a @ (b.T if tb else b)
+                if not np.array_equal(o.gemm_relu(A, B, tb, relu=False), exact.astype(float)):
+                    return False
+                if not np.array_equal(o.gemm_relu(A, B, tb, relu=True),
+                                      np.maximum(exact, 0).astype(float)):
+                    return False
+                A, B = wl.make_inputs(20, 24, 28, dtype, tb, "uniform", seed=4)
+                full = o.gemm_relu(A, B, tb)
+                r, c = wl.sample_positions(20, 24, seed=1, count=64)
+                if not np.array_equal(o.gemm_relu_sampled(A, B, r, c, tb), full[r, c]):
+                    return False
+                if not np.array_equal(o.gemm_relu_rows(A, B, [0, 7, 19], tb), full[[0, 7, 19]]):
+                    return False
+        return True
+    except Exception:
+        return False
+
+
+MUTANTS = [
+    ("last k term dropped", "for (int64_t k = 0; k < K; ++k) {\n            const double a",
+     "for (int64_t k = 0; k < K - 1; ++k) {\n            const double a"),
+    ("last k term dropped (transposed B)", "k < K; ++k) s = s + arow[k] * bcol[k];",
+     "k < K - 1; ++k) s = s + arow[k] * bcol[k];"),
+    ("relu sign flipped", "return x > 0.0 ? x : 0.0;", "return x < 0.0 ? x : 0.0;"),
+    ("trans_b branches swapped", "    if (!trans_b) {\n        for (int64_t j = j0",
+     "    if (trans_b) {\n        for (int64_t j = j0"),
+    ("fp16 exponent bias off by one", "expo - 25);", "expo - 24);"),
+    ("bf16 implicit bit dropped", "(frac | 0x80)", "(frac)"),
+    ("sampled path reads B with the other layout",
+     "trans_b ? B[j * K + k] : B[k * N + j]", "trans_b ? B[k * N + j] : B[j * K + k]"),
+]
+
+
+def test_pins_pass_on_the_real_oracle(oracle_mod):
+    assert _pins_pass(oracle_mod._default())
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_planted_mistake(oracle_mod, tmp_path, name, old, new):
+    src = open(oracle_mod._SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name!r} not unique"
+    mutant_c = tmp_path / "mutant.c"
+    mutant_c.write_text(src.replace(old, new))
+    path = oracle_mod.build(force=True, src=str(mutant_c), lib=str(tmp_path / "libmutant.so"))
+    assert not _pins_pass(oracle_mod.Oracle(path)), f"no pin caught: {name}"

@@ -1,0 +1,128 @@
+"""Seeded synthetic inputs and the named workloads of the fused GEMM + ReLU path.
+
+This module holds no arithmetic of the method itself: it only draws the
+inputs (on the host, with a CPU ``torch.Generator``) and names the shapes.
+The tests, the smoke check and the benchmark feed the same host tensors to
+the CUDA library and to the CPU oracle.
+
+Input recipe (one generator per problem, seeded with the workload's seed):
+  * A is drawn first, then B, as float32 in their stored shapes
+    (A: (M, K); B: (K, N), or (N, K) when B is stored transposed);
+  * "uniform": ``rand * 2 - 1`` (i.i.d. uniform on [-1, 1));
+    "normal": ``randn * 0.1`` (i.i.d. N(0, 1) scaled by 0.1);
+  * both are rounded to the input dtype (round-to-nearest-even, torch cast).
+
+The workloads are the matmul_relu shapes of the TileLang notes (section 3.2:
+fp16 in, fp16 out, B stored (K, N); section 3.3: bf16 in, fp32 out, B stored
+(N, K) and transposed, M = 8192 = 32 x 256, N = 7168 = 32 x 224) and the
+8192^3 FP16 GEMM the "From TVM to TileLang" essay quotes (section 3), plus
+tail and skinny shapes that exercise loop-tail handling and split-K.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import numpy as np
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    M: int
+    N: int
+    K: int
+    in_dtype: torch.dtype
+    out_dtype: torch.dtype
+    trans_b: bool
+    dist: str            # "uniform" or "normal"
+    seed: int
+    relu: bool = True
+    note: str = field(default="", compare=False)
+
+    @property
+    def flops(self) -> int:
+        """Algorithmic FLOPs: 2*M*N*K (the ReLU's M*N compares are not counted)."""
+        return 2 * self.M * self.N * self.K
+
+    @property
+    def algorithmic_bytes(self) -> int:
+        """A, B read once and C written once."""
+        isz = torch.finfo(self.in_dtype).bits // 8
+        osz = torch.finfo(self.out_dtype).bits // 8
+        return isz * (self.M * self.K + self.N * self.K) + osz * self.M * self.N
+
+
+F16, BF16, F32 = torch.float16, torch.bfloat16, torch.float32
+
+WORKLOADS = {
+    w.name: w
+    for w in [
+        Workload("square256_f16", 256, 256, 256, F16, F16, False, "uniform", 0,
+                 note="small case, the oracle finishes in well under a second"),
+        Workload("square4096_f16", 4096, 4096, 4096, F16, F16, False, "uniform", 1),
+        Workload("square8192_f16", 8192, 8192, 8192, F16, F16, False, "uniform", 2,
+                 note="the 8192^3 FP16 GEMM shape of the essay's benchmark figure"),
+        Workload("bt8192x7168x8192_bf16_f32", 8192, 7168, 8192, BF16, F32, True, "normal", 3,
+                 note="the Ascend-variant semantics: B stored (N, K), bf16 in, fp32 out"),
+        Workload("tail5000x3001x2050_f16", 5000, 3001, 2050, F16, F16, False, "uniform", 4,
+                 note="no dimension is a tile multiple and no row pitch is 16-byte aligned"),
+        Workload("skinny64x8192x8192_f16", 64, 8192, 8192, F16, F16, False, "uniform", 4,
+                 note="skinny M: memory-bound on B, split-K"),
+        Workload("skinny16x16384x4096_f16", 16, 16384, 4096, F16, F16, False, "uniform", 4,
+                 note="skinny M: memory-bound on B, split-K"),
+    ]
+}
+
+HEADLINE = "square8192_f16"
+
+
+def _draw(shape, dist: str, gen: torch.Generator) -> torch.Tensor:
+    if dist == "uniform":
+        return torch.rand(shape, generator=gen, dtype=torch.float32) * 2.0 - 1.0
+    if dist == "normal":
+        return torch.randn(shape, generator=gen, dtype=torch.float32) * 0.1
+    raise ValueError(f"unknown distribution {dist!r}")
+
+
+def make_inputs(M: int, N: int, K: int, in_dtype: torch.dtype, trans_b: bool,
+                dist: str = "uniform", seed: int = 0):
+    """Host (CPU) tensors A (M, K) and B ((N, K) if trans_b else (K, N))."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(int(seed))
+    A = _draw((M, K), dist, gen).to(in_dtype)
+    B = _draw((N, K) if trans_b else (K, N), dist, gen).to(in_dtype)
+    return A, B
+
+
+def workload_inputs(w: Workload):
+    return make_inputs(w.M, w.N, w.K, w.in_dtype, w.trans_b, w.dist, w.seed)
+
+
+def small_int_inputs(M: int, N: int, K: int, in_dtype: torch.dtype, trans_b: bool,
+                     seed: int = 0, lo: int = -4, hi: int = 4):
+    """Integer-valued inputs in [lo, hi] (exact in fp16 and bf16)."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(int(seed))
+    A = torch.randint(lo, hi + 1, (M, K), generator=gen).to(in_dtype)
+    B = torch.randint(lo, hi + 1, (N, K) if trans_b else (K, N), generator=gen).to(in_dtype)
+    return A, B
+
+
+def tile_boundaries(extent: int, tiles=(128, 256)) -> list[int]:
+    """Indices at tile edges for 128- and 256-wide tilings, plus the middle and the end."""
+    idx = {0, extent - 1, extent // 2 - 1, extent // 2}
+    for t in tiles:
+        for v in (t - 1, t, 2 * t - 1, 2 * t):
+            idx.add(v)
+        last = ((extent - 1) // t) * t
+        idx.add(last)
+        idx.add(last - 1)
+    return sorted(i for i in idx if 0 <= i < extent)
+
+
+def sample_positions(M: int, N: int, seed: int, count: int = 4096):
+    """``count`` uniformly drawn (row, col) output positions, seeded."""
+    rng = np.random.default_rng(int(seed))
+    return rng.integers(0, M, size=count, dtype=np.int64), rng.integers(0, N, size=count,
+                                                                        dtype=np.int64)
