@@ -1,0 +1,402 @@
+#!/usr/bin/env python3
+"""Benchmark of the fused GEMM + ReLU path (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference]
+
+A step is one gemm_relu call (C-ABI) over the whole workload: by default the
+8192 x 8192 x 8192 fp16 GEMM + ReLU (fp32 accumulate, fp16 out, inputs
+uniform[-1, 1] from seed 2).  Inputs are device-resident when the timed
+region starts; A + B (256 MB) exceed the 126 MB L2, so no flush is needed
+between steps.  `value` is the whole-job TFLOP/s (2*M*N*K per step per rank,
+max-over-ranks time); `e2e` repeats the measurement through the same C-ABI
+call with pinned host buffers (H2D of A and B, the call, D2H of C inside the
+timed region).
+
+Under torchrun (N > 1) each rank runs its own replica of the workload on its
+own GPU (independent problems: weak scaling, no data-path collective); the
+process group is used only for the barriers and the max over ranks.
+
+--impl reference runs the CPU oracle (the only other implementation there
+is) on a bounded sample of the same workload per step, on this host's cores.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from tiled_tensor_core_04_b200 import workloads as wl  # noqa: E402
+
+METRIC = "GEMM+ReLU TFLOP/s at 8192^3 fp16 (1 GPU), and fraction of the B200 dense tensor peak"
+PAGES_TFLOPS_8192_FP16 = 758.0  # TileLang essay, section 3 (H800): context only
+L2_BYTES = 126 * 2 ** 20
+
+# dram__bytes_read.sum + dram__bytes_write.sum per launch of the GEMM kernel,
+# from an ncu capture, keyed by the sha256 of the kernel sources it was taken
+# on (a changed kernel reports null until it is profiled again).
+NCU_TRAFFIC_BYTES: dict[str, dict[str, float]] = {}
+
+_DT = {torch.float16: "f16", torch.bfloat16: "bf16", torch.float32: "f32"}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "tiled_tensor_core_04_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0,
+            "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.period = period_s
+        self.samples: list[int] = []
+        self.reasons: set[str] = set()
+        self.max_mhz = None
+        self.error = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report it, do not guess
+            self.nvml = None
+            self.error = f"nvml unavailable: {e}"
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(
+                    self.nvml.nvmlDeviceGetClockInfo(self.handle, self.nvml.NVML_CLOCK_SM))
+                mask = self.nvml.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                for name, bit in self.REASONS.items():
+                    if mask & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception as e:
+                self.error = str(e)
+                return
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self) -> dict:
+        out = {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+               "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+               "samples": len(self.samples)}
+        if self.error:
+            out["error"] = self.error
+        return out
+
+
+# ------------------------------------------------------------------ distributed
+def dist_setup(want_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    if want_gpus != world and rank == 0:
+        print(f"warning: --gpus {want_gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ CPU oracle
+def cpu_oracle_rows(w: wl.Workload, A, B, rows) -> float:
+    """Seconds the oracle takes for the listed full output rows."""
+    import oracle
+    t0 = time.perf_counter()
+    oracle.gemm_relu_rows(A, B, rows, w.trans_b, w.relu)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(w: wl.Workload, A, B, budget_s: float = 12.0) -> dict:
+    import oracle
+    oracle.build()
+    probe = 2
+    t = cpu_oracle_rows(w, A, B, list(range(probe)))
+    rows = int(max(probe, min(1024, round(probe * budget_s / max(t, 1e-3)))))
+    rows = min(rows, w.M)
+    t = cpu_oracle_rows(w, A, B, list(range(rows)))
+    flops = 2.0 * rows * w.N * w.K
+    return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{rows} full output rows ({rows}x{w.N} of {w.M}x{w.N}) of {w.name}, "
+                      f"fp64 sequential-k sums, {t:.1f} s"}
+
+
+# ------------------------------------------------------------------ arms
+def bench_reference(args, world, rank):
+    """The CPU oracle as the reference arm (rank 0 only)."""
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    w = wl.WORKLOADS[args.workload]
+    A, B = wl.workload_inputs(w)
+    rows_per_step = max(1, args.reference_rows)
+    for i in range(args.warmup):
+        cpu_oracle_rows(w, A, B, [i % w.M])
+    times = []
+    for i in range(args.steps):
+        r = [(i * rows_per_step + j) % w.M for j in range(rows_per_step)]
+        times.append(cpu_oracle_rows(w, A, B, r))
+    total = sum(times)
+    flops = 2.0 * rows_per_step * w.N * w.K * args.steps
+    value = flops / total / 1e12
+    sample = (f"{rows_per_step} full output row(s) of {w.name} per step "
+              f"({rows_per_step}x{w.N} of {w.M}x{w.N} outputs), fp64 sequential-k sums")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, args),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w: wl.Workload, args) -> dict:
+    return {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "in_dtype": _DT[w.in_dtype],
+            "out_dtype": _DT[w.out_dtype], "trans_b": w.trans_b, "relu": w.relu,
+            "inputs": f"{w.dist}, seed {w.seed}",
+            "l2": ("inputs larger than L2 (A+B = %d MB > 126 MB), no flush"
+                   % ((w.M * w.K + w.N * w.K) * 2 // 2 ** 20))
+            if (w.M * w.K + w.N * w.K) * 2 > L2_BYTES else "L2 flushed between steps",
+            "parallelism": f"{args.gpus} independent replica(s), one per GPU"}
+
+
+def bench_ours(args, world, rank, local):
+    import tiled_tensor_core_04_b200 as g
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (there is no CPU path)")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    g.load()
+    w = wl.WORKLOADS[args.workload]
+    A_h, B_h = wl.workload_inputs(w)
+    A = A_h.to(dev)
+    B = B_h.to(dev)
+    C = torch.empty((w.M, w.N), dtype=w.out_dtype, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    sptr = stream.cuda_stream
+    props = torch.cuda.get_device_properties(dev)
+    plan = g.gemm_relu_plan(w.M, w.N, w.K, w.in_dtype, w.out_dtype, w.trans_b, A, B,
+                            num_sms=props.multi_processor_count)
+    launches_per_step = 1 + plan["pack_a"] + plan["pack_b"] + (1 if plan["split_k"] > 1 else 0)
+
+    flush = None
+    if (w.M * w.K + w.N * w.K) * torch.finfo(w.in_dtype).bits // 8 <= L2_BYTES:
+        flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        if flush is not None:
+            flush.fill_(1)
+        g.gemm_relu(A, B, C, w.M, w.N, w.K, w.in_dtype, w.out_dtype, w.trans_b, w.relu, sptr)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step()
+    torch.cuda.synchronize()
+    st, detail = g.gemm_relu_last_device_error()
+    if st != 0:
+        raise SystemExit(f"device wait ran out during warm-up (bits {detail:#x})")
+
+    # ---- device-resident timed region
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    t_begin = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    with sampler:
+        with torch.cuda.stream(stream):
+            t_begin.record(stream)
+            for i in range(args.steps):
+                if flush is not None:
+                    flush.fill_(1)
+                starts[i].record(stream)
+                g.gemm_relu(A, B, C, w.M, w.N, w.K, w.in_dtype, w.out_dtype, w.trans_b, w.relu,
+                            sptr)
+                ends[i].record(stream)
+            t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    elapsed_ms = t_begin.elapsed_time(t_end)
+    launch_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    st, detail = g.gemm_relu_last_device_error()
+    if st != 0:
+        raise SystemExit(f"device wait ran out during timing (bits {detail:#x})")
+
+    ms_per_step_local = elapsed_ms / args.steps
+    ms_per_step = max_over_ranks(ms_per_step_local, world, dev)
+    if flush is not None:  # the flush is not part of the step: time the calls only
+        ms_per_step = max_over_ranks(sum(launch_ms) / args.steps, world, dev)
+    flops = float(w.flops)
+    value = flops * world / (ms_per_step * 1e-3) / 1e12
+    kernel_ms = sum(launch_ms) / len(launch_ms)
+
+    # ---- end to end through the same call, host buffers, copies inside
+    A_pin = A_h.pin_memory()
+    B_pin = B_h.pin_memory()
+    C_pin = torch.empty((w.M, w.N), dtype=w.out_dtype).pin_memory()
+    e2e_steps = max(3, min(args.steps, args.e2e_steps))
+    with torch.cuda.stream(stream):
+        A.copy_(A_pin, non_blocking=True)
+        B.copy_(B_pin, non_blocking=True)
+        step()
+        C_pin.copy_(C, non_blocking=True)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            A.copy_(A_pin, non_blocking=True)
+            B.copy_(B_pin, non_blocking=True)
+            g.gemm_relu(A, B, C, w.M, w.N, w.K, w.in_dtype, w.out_dtype, w.trans_b, w.relu,
+                        sptr)
+            C_pin.copy_(C, non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
+    isz = torch.finfo(w.in_dtype).bits // 8
+    osz = torch.finfo(w.out_dtype).bits // 8
+
+    peaks = measured_peaks()
+    achieved = flops / (kernel_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]  # fp16 and bf16 share the dense tensor rate (ratio 1)
+    traffic = NCU_TRAFFIC_BYTES.get(kernel_source_hash(), {}).get(w.name)
+
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": value / world / PAGES_TFLOPS_8192_FP16 if w.name == wl.HEADLINE else None,
+        "dtype": _DT[w.in_dtype], "data": "synthetic", "config": workload_config(w, args),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"{peaks['source']} bf16 dense burst (fp16 same rate)",
+                     "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
+                     "kernel_ms": kernel_ms},
+        "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": isz * (w.M * w.K + w.N * w.K),
+                "d2h_bytes_per_step": osz * w.M * w.N},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": sampler.summary(),
+        "plan": {k: plan[k] for k in ("cta_pair", "tile_m", "tile_n", "tile_k", "split_k",
+                                      "units", "grid_ctas", "stages")},
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, A_h, B_h, args.cpu_budget)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=wl.HEADLINE, choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--cpu-budget", type=float, default=12.0,
+                    help="seconds of oracle work for the cpu_baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--reference-rows", type=int, default=1,
+                    help="output rows per step of the reference (CPU oracle) arm")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        # host-only arm: rank 0 runs it, the other ranks have nothing to do
+        bench_reference(args, int(os.environ.get("WORLD_SIZE", "1")),
+                        int(os.environ.get("RANK", "0")))
+        return
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        bench_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,175 @@
+/*
+ * gemm_relu.h -- C ABI of the B200 (sm_100a) fused GEMM + ReLU library.
+ *
+ *     C = relu(A . op(B))          op(B) = B  or  B^T  (trans_b)
+ *
+ * Definition followed: the matmul_relu kernel of the TileLang technical notes
+ * page, section 3.2 "GPU minimal example" (clear a fp32 accumulator,
+ * accumulate A*B over the whole K loop, take max(C, 0) element-wise, store
+ * the result), its Ascend 950 form in section 3.3 (B given as (N, K) and
+ * multiplied with transpose_B = True, bf16 in, fp32 out), and the plain
+ * tiled GEMM of the "From TVM to TileLang" essay, section 2 (relu = 0).
+ * Inputs are fp16 or bf16, products are accumulated in fp32, and the ReLU
+ * (when requested) is applied to the complete K sum before the single
+ * rounding to the output type (round-to-nearest-even).
+ *
+ * Layouts (all dense, row-major, no padding between rows):
+ *     A : M x K            element (i, k) at A[i*K + k]
+ *     B : K x N  (trans_b = 0)   element (k, j) at B[k*N + j]
+ *         N x K  (trans_b = 1)   element (k, j) at B[j*K + k]
+ *     C : M x N            element (i, j) at C[i*N + j]
+ * A and B must not overlap C.
+ *
+ * Ownership: A, B and C are DEVICE pointers owned by the caller (for
+ * example torch tensors); the caller allocates C.  The library keeps, per
+ * (device, stream), a workspace that it grows on demand with cudaMalloc and
+ * reuses: it holds fp32 split-K partial sums and, when a row pitch or base
+ * address is not 16-byte aligned (the Tensor Memory Accelerator needs
+ * 16-byte aligned rows), 16-byte-pitched copies of A and/or B.  Growing it
+ * synchronises the device; gemm_relu_release_workspace frees it.
+ *
+ * Execution: asynchronous on `stream` (a cudaStream_t passed as void*;
+ * NULL is the legacy default stream).  Nothing is synchronised; ordering
+ * with other work is stream order.  Calls on different streams of the same
+ * device may run concurrently (each stream has its own workspace).
+ *
+ * Errors: argument problems are reported synchronously by the return value
+ * and nothing is launched.  Launch failures return GEMM_ERR_CUDA (the CUDA
+ * message is kept for gemm_relu_last_cuda_error()).  Every wait inside the
+ * kernels is bounded: if one runs out (a defect, never expected), the
+ * kernel records a sticky error word on the device and returns without
+ * trapping, so the CUDA context stays usable; read it after synchronising
+ * with gemm_relu_last_device_error().  Nothing in the library aborts.
+ *
+ * Thread safety: all entry points may be called from several host threads.
+ */
+#ifndef GEMM_RELU_H_
+#define GEMM_RELU_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GEMM_RELU_API __attribute__((visibility("default")))
+#else
+#define GEMM_RELU_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GEMM_F16 = 0,  /* IEEE binary16 */
+    GEMM_BF16 = 1, /* bfloat16 */
+    GEMM_F32 = 2   /* IEEE binary32 (output only) */
+} gemm_dtype_t;
+
+typedef enum {
+    GEMM_OK = 0,
+    GEMM_ERR_INVALID_ARG = 1,       /* negative size, NULL pointer, size too large   */
+    GEMM_ERR_UNSUPPORTED_DTYPE = 2, /* in_dtype not F16/BF16, out_dtype not F16/BF16/F32 */
+    GEMM_ERR_MISALIGNED = 3,        /* reserved: misaligned operands are re-pitched, not refused */
+    GEMM_ERR_CUDA = 4,              /* a CUDA runtime/driver call failed             */
+    GEMM_ERR_TIMEOUT = 5,           /* a bounded device wait ran out (sticky word)   */
+    GEMM_ERR_NO_DEVICE = 6          /* no CUDA device, or not compute capability 10.0 */
+} gemm_status_t;
+
+/* Optional knobs.  Zero-initialise (or pass NULL) for the defaults. */
+typedef struct {
+    int cta_pair;        /* GEMM_CTA_AUTO (0), GEMM_CTA_PAIR (1), GEMM_CTA_SINGLE (2)     */
+    int split_k;         /* 0 = auto; >= 1 forces that many K splits (clamped to K/64)   */
+    int panel;           /* 0 = auto (8); >= 1 output-tile rows per L2 swizzle panel       */
+    int force_pack;      /* 1 = copy A and B through the 16-byte-pitched workspace        */
+    int max_ctas;        /* 0 = one CTA per SM; >= 1 caps the persistent grid (CTAs)      */
+    uint64_t timeout_ns; /* 0 = 1 s; bound on every in-kernel barrier wait                */
+} gemm_relu_options_t;
+/* cta_pair: 0 = auto, 1 = force the 2-CTA (256 x 256 tile, cta_group::2)
+ * kernel, 2 = force the 1-CTA (128 x 256 tile) kernel.  Split-K always uses
+ * the 1-CTA kernel. */
+#define GEMM_CTA_AUTO 0
+#define GEMM_CTA_PAIR 1
+#define GEMM_CTA_SINGLE 2
+
+/* What a call will do (filled by gemm_relu_plan). */
+typedef struct {
+    int cta_pair;        /* 1 = 2-CTA cluster kernel, 0 = 1-CTA kernel                   */
+    int tile_m, tile_n, tile_k;
+    int tiles_m, tiles_n;
+    int kblocks;         /* ceil(K / tile_k)                                              */
+    int split_k;         /* K splits per output tile (1 = none)                           */
+    int panel;
+    int units;           /* tiles_m * tiles_n * split_k work units                        */
+    int grid_ctas;       /* persistent grid size in CTAs                                  */
+    int stages;          /* shared-memory pipeline depth                                  */
+    int pack_a, pack_b;  /* 1 = operand is re-pitched into the workspace first            */
+    int64_t workspace_bytes;
+} gemm_relu_plan_t;
+
+/* C = relu(A . op(B)) (relu != 0) or A . op(B) (relu == 0).
+ * M, N, K >= 0.  M == 0 or N == 0: nothing to do, returns GEMM_OK.
+ * K == 0: C is set to zero.  trans_b selects the stored layout of B (above). */
+GEMM_RELU_API gemm_status_t gemm_relu(const void *A, const void *B, void *C,
+                        int64_t M, int64_t N, int64_t K,
+                        gemm_dtype_t in_dtype, gemm_dtype_t out_dtype,
+                        int trans_b, int relu, void *stream);
+
+/* Same, with explicit options (NULL = defaults). */
+GEMM_RELU_API gemm_status_t gemm_relu_ex(const void *A, const void *B, void *C,
+                           int64_t M, int64_t N, int64_t K,
+                           gemm_dtype_t in_dtype, gemm_dtype_t out_dtype,
+                           int trans_b, int relu, void *stream,
+                           const gemm_relu_options_t *opts);
+
+/* The plan a call with these arguments would use, computed on the host only
+ * (no GPU needed).  num_sms: SMs of the target device (148 on B200);
+ * max_pair_clusters: how many 2-CTA clusters fit at once (0 = num_sms / 2).
+ * A and B are used only for their address alignment (NULL = aligned). */
+GEMM_RELU_API gemm_status_t gemm_relu_plan(int64_t M, int64_t N, int64_t K,
+                             gemm_dtype_t in_dtype, gemm_dtype_t out_dtype, int trans_b,
+                             const void *A, const void *B,
+                             int num_sms, int max_pair_clusters,
+                             const gemm_relu_options_t *opts, gemm_relu_plan_t *plan);
+
+/* One work unit of a plan: output tile (tile_row, tile_col) and the K
+ * blocks [kb_begin, kb_end) it accumulates (split index `split`). */
+typedef struct {
+    int tile_row, tile_col, kb_begin, kb_end, split;
+} gemm_relu_unit_t;
+
+/* The unit the persistent kernels process as number `u` (0 <= u < units):
+ * the same tile walk the device uses (panels of `panel` tile rows, column by
+ * column inside a panel, splits of one tile adjacent).  Host only. */
+GEMM_RELU_API gemm_status_t gemm_relu_plan_unit(const gemm_relu_plan_t *plan, int u,
+                                                gemm_relu_unit_t *unit);
+
+/* Static description of a status code (never NULL). */
+GEMM_RELU_API const char *gemm_relu_status_string(gemm_status_t status);
+
+/* Message of the last CUDA error seen by this host thread ("" if none). */
+GEMM_RELU_API const char *gemm_relu_last_cuda_error(void);
+
+/* Reads and clears the sticky device error word of the current device.
+ * Synchronises the device.  GEMM_OK if no bounded wait has run out since the
+ * last read, GEMM_ERR_TIMEOUT otherwise; *detail (if not NULL) receives the
+ * raw bit mask of which waits gave up (1 producer slot, 2 MMA operands,
+ * 4 MMA accumulator, 8 epilogue accumulator, 16 teardown drain, 32 self-test). */
+GEMM_RELU_API gemm_status_t gemm_relu_last_device_error(uint32_t *detail);
+
+/* Failure-detection self-test: launches one tiny kernel whose threads wait on
+ * an mbarrier that nothing ever arrives on, bounded by timeout_ns, and
+ * synchronises.  Returns GEMM_ERR_TIMEOUT when the wait ran out and was
+ * reported as designed (the context stays usable), GEMM_OK if the wait
+ * unexpectedly completed, another code on a CUDA failure.  The device error
+ * word is left set (bit 32) for gemm_relu_last_device_error to read. */
+GEMM_RELU_API gemm_status_t gemm_relu_selftest_timeout(uint64_t timeout_ns, void *stream);
+
+/* Frees this process's workspaces on the current device (synchronises it). */
+GEMM_RELU_API gemm_status_t gemm_relu_release_workspace(void);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+GEMM_RELU_API int gemm_relu_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GEMM_RELU_H_ */

@@ -1,0 +1,170 @@
+"""The C-ABI library on the CPU (no GPU): it loads, exports every symbol the
+header declares, plans every workload as designed, walks every (tile, K
+block) exactly once, and rejects bad arguments without launching anything.
+"""
+from __future__ import annotations
+
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+import tiled_tensor_core_04_b200 as g
+from tiled_tensor_core_04_b200 import build as gbuild
+from tiled_tensor_core_04_b200 import workloads as wl
+
+HEADER = os.path.join(gbuild.ROOT, "include", "gemm_relu.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    gbuild.build()
+    return g.load()
+
+
+def header_functions() -> set[str]:
+    text = open(HEADER).read()
+    return set(re.findall(r"GEMM_RELU_API\s+[\w\s\*]*?\b(gemm_relu\w*)\s*\(", text))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    declared = header_functions()
+    assert declared == set(g.EXPORTS)
+    out = subprocess.run(["nm", "-D", "--defined-only", gbuild.LIB], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    assert declared <= exported, declared - exported
+    for name in declared:
+        assert hasattr(lib, name)
+
+
+def test_library_is_sm100a_only():
+    # the build flags name exactly one target: sm_100a
+    flags = " ".join(gbuild.NVCC_FLAGS)
+    assert "arch=compute_100a,code=sm_100a" in flags
+    assert flags.count("arch=") == 1
+
+
+def test_version_and_status_strings(lib):
+    assert g.gemm_relu_version() == 10000
+    for code in range(7):
+        assert g.gemm_relu_status_string(code)
+    assert g.gemm_relu_status_string(99) == "unknown status"
+
+
+def plan(w: wl.Workload, **opt):
+    return g.gemm_relu_plan(w.M, w.N, w.K, w.in_dtype, w.out_dtype, w.trans_b,
+                            options=opt or None)
+
+
+def test_plans_for_the_workloads(lib):
+    p = plan(wl.WORKLOADS["square8192_f16"])
+    assert (p["cta_pair"], p["tile_m"], p["tile_n"], p["split_k"]) == (1, 256, 256, 1)
+    assert (p["tiles_m"], p["tiles_n"], p["units"], p["grid_ctas"]) == (32, 32, 1024, 148)
+    assert p["pack_a"] == p["pack_b"] == 0 and p["workspace_bytes"] == 0
+
+    p = plan(wl.WORKLOADS["bt8192x7168x8192_bf16_f32"])
+    assert p["cta_pair"] == 1 and p["tiles_n"] == 28 and p["units"] == 896
+
+    p = plan(wl.WORKLOADS["tail5000x3001x2050_f16"])
+    assert p["pack_a"] == 1 and p["pack_b"] == 1          # 4100- and 6002-byte row pitches
+    assert p["kblocks"] == 33 and p["tiles_m"] == 20 and p["tiles_n"] == 12
+
+    p = plan(wl.WORKLOADS["skinny64x8192x8192_f16"])
+    assert p["cta_pair"] == 0 and p["split_k"] == 4 and p["units"] == 128
+    assert p["workspace_bytes"] >= 4 * 64 * 8192 * 4
+
+    p = plan(wl.WORKLOADS["skinny16x16384x4096_f16"])
+    assert p["cta_pair"] == 0 and p["split_k"] == 2 and p["units"] == 128
+
+    p = plan(wl.WORKLOADS["square256_f16"])
+    assert p["units"] == 1 and p["grid_ctas"] == 2
+
+
+def test_options_override_the_plan(lib):
+    w = wl.WORKLOADS["square4096_f16"]
+    assert plan(w, cta_pair=g.GEMM_CTA_SINGLE)["cta_pair"] == 0
+    assert plan(w, cta_pair=g.GEMM_CTA_PAIR)["cta_pair"] == 1
+    p = plan(w, split_k=3)
+    assert p["split_k"] == 3 and p["cta_pair"] == 0
+    assert plan(w, split_k=10 ** 6)["split_k"] == 64        # clamped to K / 64
+    assert plan(w, max_ctas=10)["grid_ctas"] == 10
+    assert plan(w, max_ctas=10, cta_pair=g.GEMM_CTA_PAIR)["grid_ctas"] == 10
+    assert plan(w, force_pack=1)["pack_a"] == 1
+    assert plan(w, panel=3)["panel"] == 3
+
+
+def test_misaligned_base_pointer_is_repitched(lib):
+    p = g.gemm_relu_plan(512, 512, 512, torch.float16, torch.float16, False, A=0x1002, B=0x2000)
+    assert p["pack_a"] == 1 and p["pack_b"] == 0
+    p = g.gemm_relu_plan(512, 512, 512, torch.float16, torch.float16, True, A=0x1000, B=0x2008)
+    assert p["pack_a"] == 0 and p["pack_b"] == 1
+
+
+@pytest.mark.parametrize("M,N,K,opt", [
+    (8192, 8192, 8192, {}),
+    (5000, 3001, 2050, {}),
+    (64, 8192, 8192, {}),
+    (300, 700, 1000, {"split_k": 7, "panel": 3}),
+    (1000, 300, 130, {"cta_pair": g.GEMM_CTA_SINGLE, "panel": 5}),
+    (257, 257, 65, {"panel": 1}),
+])
+def test_units_cover_every_tile_and_k_block_once(lib, M, N, K, opt):
+    p = g.gemm_relu_plan(M, N, K, torch.float16, torch.float16, False, options=opt or None)
+    seen = {}
+    for u in range(p["units"]):
+        r, c, kb0, kb1, s = g.gemm_relu_plan_unit(p, u)
+        assert 0 <= r < p["tiles_m"] and 0 <= c < p["tiles_n"] and 0 <= s < p["split_k"]
+        assert 0 <= kb0 < kb1 <= p["kblocks"]
+        seen.setdefault((r, c), []).append((kb0, kb1, s))
+    assert len(seen) == p["tiles_m"] * p["tiles_n"]
+    for spans in seen.values():
+        spans.sort()
+        assert [s for _, _, s in spans] == list(range(p["split_k"]))
+        assert spans[0][0] == 0 and spans[-1][1] == p["kblocks"]
+        assert all(a[1] == b[0] for a, b in zip(spans, spans[1:]))
+
+
+def test_panel_swizzle_keeps_consecutive_units_in_a_panel(lib):
+    p = g.gemm_relu_plan(8192, 8192, 8192, torch.float16, torch.float16, False)
+    rows = [g.gemm_relu_plan_unit(p, u)[0] for u in range(p["grid_ctas"] // 2)]
+    assert set(rows) == set(range(8))                      # one panel of 8 tile rows
+    cols = [g.gemm_relu_plan_unit(p, u)[1] for u in range(p["grid_ctas"] // 2)]
+    assert max(cols) == (p["grid_ctas"] // 2 - 1) // 8
+
+
+@pytest.mark.parametrize("args,status", [
+    ((-1, 4, 4, 0, 0), g.GEMM_ERR_INVALID_ARG),
+    ((4, -1, 4, 0, 0), g.GEMM_ERR_INVALID_ARG),
+    ((4, 4, -1, 0, 0), g.GEMM_ERR_INVALID_ARG),
+    ((2 ** 31, 4, 4, 0, 0), g.GEMM_ERR_INVALID_ARG),
+    ((4, 4, 4, 2, 0), g.GEMM_ERR_UNSUPPORTED_DTYPE),      # fp32 inputs
+    ((4, 4, 4, 0, 7), g.GEMM_ERR_UNSUPPORTED_DTYPE),
+])
+def test_bad_arguments_are_refused_before_any_launch(lib, args, status):
+    M, N, K, din, dout = args
+    st = g.gemm_relu(0x1000, 0x2000, 0x3000, M, N, K, din, dout, 0, 1, 0, check=False)
+    assert st == status
+    with pytest.raises(g.GemmError):
+        g.gemm_relu_plan(M, N, K, din, dout, 0)
+
+
+def test_null_pointers_and_empty_problems(lib):
+    assert g.gemm_relu(0, 0x2000, 0x3000, 4, 4, 4, 0, 0, 0, 1, 0, check=False) == \
+        g.GEMM_ERR_INVALID_ARG
+    assert g.gemm_relu(0x1000, 0x2000, 0, 4, 4, 4, 0, 0, 0, 1, 0, check=False) == \
+        g.GEMM_ERR_INVALID_ARG
+    # nothing to compute: returns before touching any device
+    assert g.gemm_relu(0, 0, 0, 0, 5, 5, 0, 0, 0, 1, 0, check=False) == g.GEMM_OK
+    assert g.gemm_relu(0, 0, 0, 5, 0, 5, 0, 0, 0, 1, 0, check=False) == g.GEMM_OK
+    with pytest.raises(KeyError):
+        g.gemm_relu_ex(0, 0, 0, 0, 0, 0, 0, 0, 0, 1, 0, options={"bogus": 1})
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU answer")
+def test_no_device_is_reported_not_faked(lib):
+    st = g.gemm_relu(0x1000, 0x2000, 0x3000, 4, 4, 4, 0, 0, 0, 1, 0, check=False)
+    assert st == g.GEMM_ERR_NO_DEVICE
+    assert g.gemm_relu_selftest_timeout(1000000) == g.GEMM_ERR_NO_DEVICE

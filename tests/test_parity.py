@@ -1,0 +1,251 @@
+"""GPU parity: the sm_100a library against the CPU oracle, element by element.
+
+All calls go through the C ABI (ctypes binding).  Inputs are the seeded
+host tensors of tiled_tensor_core_04_b200.workloads, copied to the device;
+the oracle sees the same host tensors.  Tolerances are those of
+tests/parity_util.py (fp16 out: 1e-2 + 2e-3|ref|, fp32 out: 1e-3 + 1e-4|ref|,
+bf16 out: 1e-2 + 4e-3|ref|), against the unrounded fp64 oracle value.
+
+Every output buffer sits inside a larger allocation pre-filled with NaN: the
+test checks that exactly the M x N result was written and nothing after it.
+After every call the sticky device error word must be clear.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import tiled_tensor_core_04_b200 as g
+from tests.parity_util import check_close
+from tiled_tensor_core_04_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+F16, BF16, F32 = torch.float16, torch.bfloat16, torch.float32
+PAD = 4096  # guard elements after C
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    g.load()
+    oracle.build()
+    yield
+    torch.cuda.synchronize()
+
+
+def device_error_clear():
+    st, detail = g.gemm_relu_last_device_error()
+    assert st == g.GEMM_OK, f"device wait ran out (bits {detail:#x})"
+
+
+def run(A: torch.Tensor, B: torch.Tensor, out_dtype, trans_b: bool, relu: bool = True,
+        options=None, c_offset: int = 0, a_offset: int = 0, stream=None):
+    """Call the library on device copies of A, B; return C on the host."""
+    M, K = A.shape
+    N = B.shape[0] if trans_b else B.shape[1]
+    dev = torch.device("cuda")
+    if a_offset:
+        abuf = torch.empty(A.numel() + a_offset, dtype=A.dtype, device=dev)
+        Ad = abuf[a_offset:].view(M, K)
+        Ad.copy_(A)
+    else:
+        Ad = A.to(dev)
+    Bd = B.to(dev)
+    cbuf = torch.full((M * N + PAD + c_offset,), float("nan"), dtype=out_dtype, device=dev)
+    Cd = cbuf[c_offset:c_offset + M * N].view(M, N)
+    g.gemm_relu_ex(Ad, Bd, Cd, M, N, K, A.dtype, out_dtype, trans_b, relu,
+                   stream=stream, options=options)
+    torch.cuda.synchronize()
+    device_error_clear()
+    tail = cbuf[c_offset + M * N:].float().cpu()
+    assert torch.isnan(tail).all(), "wrote past the end of C"
+    if c_offset:
+        assert torch.isnan(cbuf[:c_offset].float().cpu()).all(), "wrote before C"
+    return Cd.cpu()
+
+
+def full_case(M, N, K, in_dtype, out_dtype, trans_b, relu=True, options=None, seed=0,
+              dist="uniform", **kw):
+    A, B = wl.make_inputs(M, N, K, in_dtype, trans_b, dist, seed)
+    C = run(A, B, out_dtype, trans_b, relu, options, **kw)
+    ref = oracle.gemm_relu(A, B, trans_b=trans_b, relu=relu)
+    return check_close(C, ref, out_dtype, relu, what=f"{M}x{N}x{K}")
+
+
+# ---------------------------------------------------------------- full oracle
+SHAPES = [
+    (128, 256, 64),      # exactly one 1-CTA tile, one K block
+    (256, 256, 256),     # one pair tile
+    (129, 257, 65),      # one past every tile edge
+    (300, 520, 200),
+    (513, 768, 1000),
+    (1000, 300, 130),
+    (64, 8, 8),          # smallest 16-byte-aligned N
+    (1, 1, 1),           # everything re-pitched, one element
+    (3, 5, 7),
+    (37, 1000, 24),
+]
+
+VARIANTS = {
+    "auto": None,
+    "single": {"cta_pair": g.GEMM_CTA_SINGLE},
+    "pair": {"cta_pair": g.GEMM_CTA_PAIR},
+    "split3": {"split_k": 3},
+    "packed": {"force_pack": 1},
+    "few_ctas": {"max_ctas": 3, "panel": 2},
+}
+
+
+@pytest.mark.parametrize("variant", list(VARIANTS))
+@pytest.mark.parametrize("trans_b", [False, True])
+@pytest.mark.parametrize("M,N,K", SHAPES)
+def test_shapes_fp16(M, N, K, trans_b, variant):
+    full_case(M, N, K, F16, F16, trans_b, options=VARIANTS[variant], seed=M + N + K)
+
+
+@pytest.mark.parametrize("out_dtype", [F16, BF16, F32])
+@pytest.mark.parametrize("in_dtype", [F16, BF16])
+@pytest.mark.parametrize("trans_b", [False, True])
+@pytest.mark.parametrize("relu", [True, False])
+@pytest.mark.parametrize("variant", ["auto", "single", "split3"])
+def test_dtypes_and_relu(in_dtype, out_dtype, trans_b, relu, variant):
+    full_case(300, 520, 330, in_dtype, out_dtype, trans_b, relu, VARIANTS[variant], seed=7,
+              dist="normal")
+
+
+def test_square256_full():
+    w = wl.WORKLOADS["square256_f16"]
+    A, B = wl.workload_inputs(w)
+    C = run(A, B, w.out_dtype, w.trans_b)
+    check_close(C, oracle.gemm_relu(A, B, w.trans_b), w.out_dtype, True, w.name)
+
+
+@pytest.mark.parametrize("name", ["tail5000x3001x2050_f16", "skinny64x8192x8192_f16",
+                                  "skinny16x16384x4096_f16"])
+def test_tail_and_skinny_workloads_full(name):
+    w = wl.WORKLOADS[name]
+    A, B = wl.workload_inputs(w)
+    C = run(A, B, w.out_dtype, w.trans_b)
+    check_close(C, oracle.gemm_relu(A, B, w.trans_b), w.out_dtype, True, w.name)
+
+
+# ---------------------------------------------------------------- full size, sampled
+def sampled_check(w: wl.Workload, C: torch.Tensor, A, B):
+    rows, cols = wl.sample_positions(w.M, w.N, seed=w.seed + 1000, count=4096)
+    ref = oracle.gemm_relu_sampled(A, B, rows, cols, w.trans_b)
+    got = C[torch.from_numpy(rows), torch.from_numpy(cols)]
+    check_close(got, ref, w.out_dtype, True, f"{w.name} sampled")
+    br = wl.tile_boundaries(w.M)
+    check_close(C[br], oracle.gemm_relu_rows(A, B, br, w.trans_b), w.out_dtype, True,
+                f"{w.name} boundary rows")
+    bc = wl.tile_boundaries(w.N)
+    check_close(C[:, bc], oracle.gemm_relu_cols(A, B, bc, w.trans_b), w.out_dtype, True,
+                f"{w.name} boundary cols")
+
+
+@pytest.mark.parametrize("name", ["square4096_f16", "square8192_f16",
+                                  "bt8192x7168x8192_bf16_f32"])
+def test_full_size_workloads_sampled(name):
+    w = wl.WORKLOADS[name]
+    A, B = wl.workload_inputs(w)
+    C = run(A, B, w.out_dtype, w.trans_b)
+    assert torch.isfinite(C.float()).all() and (C.float() >= 0).all()
+    sampled_check(w, C, A, B)
+
+
+# ---------------------------------------------------------------- closed forms
+@pytest.mark.parametrize("variant", ["auto", "single", "split3"])
+@pytest.mark.parametrize("trans_b", [False, True])
+@pytest.mark.parametrize("M,N,K", [(300, 520, 2050), (256, 512, 8192), (70, 33, 9)])
+def test_ones_give_exactly_K(M, N, K, trans_b, variant):
+    A = torch.ones(M, K, dtype=F16)
+    B = torch.ones((N, K) if trans_b else (K, N), dtype=F16)
+    C = run(A, B, F16, trans_b, True, VARIANTS[variant])
+    assert (C.float() == K).all()          # K = 2050, 8192, 9 are exact in fp16
+
+
+@pytest.mark.parametrize("trans_b", [False, True])
+@pytest.mark.parametrize("relu", [False, True])
+@pytest.mark.parametrize("in_dtype", [F16, BF16])
+def test_identity_gives_relu_A(trans_b, relu, in_dtype):
+    M, K = 333, 320
+    A, _ = wl.make_inputs(M, K, K, in_dtype, False, "uniform", seed=5)
+    B = torch.eye(K, dtype=in_dtype)
+    C = run(A, B, in_dtype, trans_b, relu)
+    want = A.clamp_min(0) if relu else A
+    assert torch.equal(C, want)
+
+
+@pytest.mark.parametrize("trans_b", [False, True])
+def test_all_negative_product_is_zero(trans_b):
+    A, B = wl.make_inputs(200, 300, 500, F16, trans_b, "uniform", seed=6)
+    C = run(A.abs(), -B.abs(), F16, trans_b, True)
+    assert (C.float() == 0).all()
+
+
+@pytest.mark.parametrize("variant", ["auto", "single", "split3", "packed"])
+@pytest.mark.parametrize("trans_b", [False, True])
+@pytest.mark.parametrize("in_dtype", [F16, BF16])
+@pytest.mark.parametrize("M,N,K", [(300, 520, 1000), (129, 264, 72), (5000 // 8, 3001, 2050)])
+def test_small_integers_bit_exact(M, N, K, in_dtype, trans_b, variant):
+    A, B = wl.small_int_inputs(M, N, K, in_dtype, trans_b, seed=M)
+    exact = A.to(torch.int64) @ (B.to(torch.int64).t() if trans_b else B.to(torch.int64))
+    C = run(A, B, F32, trans_b, True, VARIANTS[variant])
+    assert torch.equal(C.to(torch.int64), exact.clamp_min(0))
+    assert torch.equal(C, exact.clamp_min(0).to(F32))
+
+
+# ---------------------------------------------------------------- edges
+def test_K_zero_writes_zeros():
+    A = torch.zeros(70, 0, dtype=F16)
+    B = torch.zeros(0, 90, dtype=F16)
+    C = run(A, B, F16, False)
+    assert (C.float() == 0).all()
+
+
+def test_M_or_N_zero_is_a_no_op():
+    dev = torch.device("cuda")
+    A = torch.ones(0, 64, dtype=F16, device=dev)
+    B = torch.ones(64, 64, dtype=F16, device=dev)
+    C = torch.full((4,), 7.0, dtype=F16, device=dev)
+    g.gemm_relu(A, B, C, 0, 64, 64, F16, F16, False, True)
+    g.gemm_relu(B, A, C, 64, 0, 64, F16, F16, True, True)
+    torch.cuda.synchronize()
+    assert (C.float() == 7).all()
+
+
+@pytest.mark.parametrize("c_offset,a_offset", [(1, 0), (0, 1), (3, 5)])
+def test_misaligned_pointers(c_offset, a_offset):
+    full_case(260, 264, 136, F16, F16, False, c_offset=c_offset, a_offset=a_offset, seed=9)
+
+
+def test_runs_are_deterministic():
+    A, B = wl.make_inputs(64, 4096, 4096, F16, False, "uniform", seed=11)
+    c1 = run(A, B, F16, False)
+    c2 = run(A, B, F16, False)
+    assert torch.equal(c1, c2)
+    A, B = wl.make_inputs(700, 900, 1500, F16, True, "uniform", seed=12)
+    assert torch.equal(run(A, B, F32, True), run(A, B, F32, True))
+
+
+def test_side_stream_and_matmul_relu_helper():
+    A, B = wl.make_inputs(300, 400, 500, F16, False, "uniform", seed=13)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        Ad, Bd = A.cuda(), B.cuda()
+        C = g.matmul_relu(Ad, Bd)
+    s.synchronize()
+    device_error_clear()
+    check_close(C.cpu(), oracle.gemm_relu(A, B), F16, True, "side stream")
+
+
+def test_headline_plan_is_the_pair_kernel():
+    w = wl.WORKLOADS[wl.HEADLINE]
+    props = torch.cuda.get_device_properties(0)
+    p = g.gemm_relu_plan(w.M, w.N, w.K, w.in_dtype, w.out_dtype, w.trans_b,
+                         num_sms=props.multi_processor_count)
+    assert p["cta_pair"] == 1 and p["split_k"] == 1

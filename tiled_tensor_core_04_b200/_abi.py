@@ -1,0 +1,247 @@
+"""ctypes binding of the C ABI in include/gemm_relu.h (argument marshalling only).
+
+Every computation runs in libgemmrelu.so (CUDA, sm_100a).  There is no CPU or
+PyTorch fallback: if the library is missing or the device is not a
+compute-capability 10.0 GPU, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgemmrelu.so")
+
+GEMM_F16, GEMM_BF16, GEMM_F32 = 0, 1, 2
+GEMM_CTA_AUTO, GEMM_CTA_PAIR, GEMM_CTA_SINGLE = 0, 1, 2
+
+STATUS = {
+    0: "GEMM_OK",
+    1: "GEMM_ERR_INVALID_ARG",
+    2: "GEMM_ERR_UNSUPPORTED_DTYPE",
+    3: "GEMM_ERR_MISALIGNED",
+    4: "GEMM_ERR_CUDA",
+    5: "GEMM_ERR_TIMEOUT",
+    6: "GEMM_ERR_NO_DEVICE",
+}
+GEMM_OK, GEMM_ERR_INVALID_ARG, GEMM_ERR_UNSUPPORTED_DTYPE = 0, 1, 2
+GEMM_ERR_MISALIGNED, GEMM_ERR_CUDA, GEMM_ERR_TIMEOUT, GEMM_ERR_NO_DEVICE = 3, 4, 5, 6
+
+# every symbol the header declares
+EXPORTS = (
+    "gemm_relu", "gemm_relu_ex", "gemm_relu_plan", "gemm_relu_status_string",
+    "gemm_relu_last_cuda_error", "gemm_relu_last_device_error", "gemm_relu_selftest_timeout",
+    "gemm_relu_release_workspace", "gemm_relu_version", "gemm_relu_plan_unit",
+)
+
+_DTYPE_CODE = {torch.float16: GEMM_F16, torch.bfloat16: GEMM_BF16, torch.float32: GEMM_F32}
+
+
+class GemmOptions(ctypes.Structure):
+    _fields_ = [
+        ("cta_pair", ctypes.c_int),
+        ("split_k", ctypes.c_int),
+        ("panel", ctypes.c_int),
+        ("force_pack", ctypes.c_int),
+        ("max_ctas", ctypes.c_int),
+        ("timeout_ns", ctypes.c_uint64),
+    ]
+
+
+class GemmPlan(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in (
+        "cta_pair", "tile_m", "tile_n", "tile_k", "tiles_m", "tiles_n", "kblocks", "split_k",
+        "panel", "units", "grid_ctas", "stages", "pack_a", "pack_b")] + [
+        ("workspace_bytes", ctypes.c_int64)]
+
+    def as_dict(self) -> dict:
+        return {n: getattr(self, n) for n, _ in self._fields_}
+
+
+class GemmUnit(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("tile_row", "tile_col", "kb_begin", "kb_end", "split")]
+
+
+class GemmError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def load():
+    """Load libgemmrelu.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise ImportError(
+                    f"CUDA library {LIB_PATH} is missing; build it with "
+                    "`python -m tiled_tensor_core_04_b200.build` (there is no fallback)")
+            lib = ctypes.CDLL(LIB_PATH)
+            i64, i32, vp, u64 = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_uint64
+            gemm_args = [vp, vp, vp, i64, i64, i64, i32, i32, i32, i32, vp]
+            lib.gemm_relu.argtypes = gemm_args
+            lib.gemm_relu_ex.argtypes = gemm_args + [ctypes.POINTER(GemmOptions)]
+            lib.gemm_relu_plan.argtypes = [i64, i64, i64, i32, i32, i32, vp, vp, i32, i32,
+                                           ctypes.POINTER(GemmOptions), ctypes.POINTER(GemmPlan)]
+            lib.gemm_relu_plan_unit.argtypes = [ctypes.POINTER(GemmPlan), i32,
+                                                ctypes.POINTER(GemmUnit)]
+            lib.gemm_relu_status_string.argtypes = [i32]
+            lib.gemm_relu_status_string.restype = ctypes.c_char_p
+            lib.gemm_relu_last_cuda_error.argtypes = []
+            lib.gemm_relu_last_cuda_error.restype = ctypes.c_char_p
+            lib.gemm_relu_last_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
+            lib.gemm_relu_selftest_timeout.argtypes = [u64, vp]
+            lib.gemm_relu_release_workspace.argtypes = []
+            lib.gemm_relu_version.argtypes = []
+            for name in ("gemm_relu", "gemm_relu_ex", "gemm_relu_plan", "gemm_relu_last_device_error",
+                         "gemm_relu_selftest_timeout", "gemm_relu_release_workspace",
+                         "gemm_relu_version", "gemm_relu_plan_unit"):
+                getattr(lib, name).restype = i32
+            _lib = lib
+    return _lib
+
+
+# ------------------------------------------------------------------ marshalling
+def _ptr(x) -> int:
+    if x is None:
+        return 0
+    if isinstance(x, torch.Tensor):
+        return x.data_ptr()
+    return int(x)
+
+
+def _dtype(x) -> int:
+    if isinstance(x, torch.dtype):
+        if x not in _DTYPE_CODE:
+            return 99  # rejected by the library as unsupported
+        return _DTYPE_CODE[x]
+    return int(x)
+
+
+def _stream(s) -> int:
+    if s is None:
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else 0
+    if isinstance(s, torch.cuda.Stream):
+        return s.cuda_stream
+    return int(s)
+
+
+def _options(opts) -> GemmOptions | None:
+    if opts is None:
+        return None
+    if isinstance(opts, GemmOptions):
+        return opts
+    o = GemmOptions()
+    for k, v in dict(opts).items():
+        if not hasattr(o, k):
+            raise KeyError(f"unknown option {k!r}")
+        setattr(o, k, int(v))
+    return o
+
+
+def _check(status: int) -> int:
+    if status != GEMM_OK:
+        lib = load()
+        msg = lib.gemm_relu_status_string(status).decode()
+        cuda = lib.gemm_relu_last_cuda_error().decode()
+        raise GemmError(status, msg + (f" ({cuda})" if cuda else ""))
+    return status
+
+
+def gemm_relu(A, B, C, M, N, K, in_dtype, out_dtype, trans_b, relu, stream=None,
+              check: bool = True) -> int:
+    """The C entry point; pointers may be ints or tensors, dtypes codes or torch dtypes."""
+    st = load().gemm_relu(_ptr(A), _ptr(B), _ptr(C), int(M), int(N), int(K), _dtype(in_dtype),
+                          _dtype(out_dtype), int(bool(trans_b)), int(bool(relu)),
+                          _stream(stream))
+    return _check(st) if check else st
+
+
+def gemm_relu_ex(A, B, C, M, N, K, in_dtype, out_dtype, trans_b, relu, stream=None,
+                 options=None, check: bool = True) -> int:
+    o = _options(options)
+    st = load().gemm_relu_ex(_ptr(A), _ptr(B), _ptr(C), int(M), int(N), int(K), _dtype(in_dtype),
+                             _dtype(out_dtype), int(bool(trans_b)), int(bool(relu)),
+                             _stream(stream), ctypes.byref(o) if o is not None else None)
+    return _check(st) if check else st
+
+
+def gemm_relu_plan(M, N, K, in_dtype, out_dtype, trans_b, A=None, B=None, num_sms=148,
+                   max_pair_clusters=0, options=None) -> dict:
+    o = _options(options)
+    plan = GemmPlan()
+    st = load().gemm_relu_plan(int(M), int(N), int(K), _dtype(in_dtype), _dtype(out_dtype),
+                               int(bool(trans_b)), _ptr(A), _ptr(B), int(num_sms),
+                               int(max_pair_clusters), ctypes.byref(o) if o is not None else None,
+                               ctypes.byref(plan))
+    _check(st)
+    return plan.as_dict()
+
+
+def gemm_relu_plan_unit(plan: dict, u: int) -> tuple[int, int, int, int, int]:
+    """(tile_row, tile_col, kb_begin, kb_end, split) of work unit `u` of a plan dict."""
+    p = GemmPlan(**{k: plan[k] for k, _ in GemmPlan._fields_})
+    unit = GemmUnit()
+    _check(load().gemm_relu_plan_unit(ctypes.byref(p), int(u), ctypes.byref(unit)))
+    return unit.tile_row, unit.tile_col, unit.kb_begin, unit.kb_end, unit.split
+
+
+def gemm_relu_status_string(status: int) -> str:
+    return load().gemm_relu_status_string(int(status)).decode()
+
+
+def gemm_relu_last_cuda_error() -> str:
+    return load().gemm_relu_last_cuda_error().decode()
+
+
+def gemm_relu_last_device_error() -> tuple[int, int]:
+    """(status, detail bits); reads and clears the sticky device error word."""
+    detail = ctypes.c_uint32(0)
+    st = load().gemm_relu_last_device_error(ctypes.byref(detail))
+    return st, int(detail.value)
+
+
+def gemm_relu_selftest_timeout(timeout_ns: int, stream=None) -> int:
+    return load().gemm_relu_selftest_timeout(int(timeout_ns), _stream(stream))
+
+
+def gemm_relu_release_workspace() -> int:
+    return _check(load().gemm_relu_release_workspace())
+
+
+def gemm_relu_version() -> int:
+    return int(load().gemm_relu_version())
+
+
+# ------------------------------------------------------------------ tensor helper
+def matmul_relu(A: torch.Tensor, B: torch.Tensor, trans_b: bool = False, relu: bool = True,
+                out_dtype: torch.dtype | None = None, out: torch.Tensor | None = None,
+                stream=None, options=None) -> torch.Tensor:
+    """C = relu(A @ op(B)) on CUDA tensors; allocates C (torch) unless `out` is given."""
+    if A.dim() != 2 or B.dim() != 2:
+        raise ValueError("A and B must be 2-D")
+    if not (A.is_cuda and B.is_cuda):
+        raise ValueError("A and B must be CUDA tensors (no CPU path)")
+    if not (A.is_contiguous() and B.is_contiguous()):
+        raise ValueError("A and B must be contiguous row-major")
+    M, K = A.shape
+    N = B.shape[0] if trans_b else B.shape[1]
+    if (B.shape[1] if trans_b else B.shape[0]) != K:
+        raise ValueError("inner dimensions differ")
+    if A.dtype != B.dtype:
+        raise TypeError("A and B must have the same dtype")
+    out_dtype = out_dtype or A.dtype
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=A.device)
+    elif out.shape != (M, N) or out.dtype != out_dtype or not out.is_contiguous():
+        raise ValueError("out must be a contiguous (M, N) tensor of out_dtype")
+    gemm_relu_ex(A, B, out, M, N, K, A.dtype, out_dtype, trans_b, relu, stream, options)
+    return out

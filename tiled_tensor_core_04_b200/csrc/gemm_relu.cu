@@ -1,0 +1,590 @@
+// gemm_relu.cu -- host side of the C ABI declared in include/gemm_relu.h:
+// argument checks, the launch plan (tile shape, CTA pair or single, split-K,
+// re-pitching), the per-stream workspace, TMA tensor-map encoding, and the
+// kernel launches.  All device work is in gemm_kernel.cuh / aux_kernels.cuh.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <utility>
+
+#include "../../include/gemm_relu.h"
+#include "aux_kernels.cuh"
+#include "gemm_kernel.cuh"
+
+namespace {
+
+using namespace gr;
+
+constexpr int kVersion = 10000;  // 1.0.0
+constexpr uint64_t kDefaultTimeoutNs = 1000000000ull;  // 1 s per barrier wait
+constexpr int kDefaultPanel = 8;
+constexpr int kMaxDevices = 64;
+
+thread_local std::string t_last_cuda_error;
+
+gemm_status_t cuda_fail(cudaError_t e, const char *what)
+{
+    t_last_cuda_error = std::string(what) + ": " + cudaGetErrorString(e);
+    return GEMM_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ kernels
+using GemmKernelFn = void (*)(const CUtensorMap, const CUtensorMap, const GemmParams);
+
+template <bool PAIR, bool BMN>
+GemmKernelFn pick_out(gemm_dtype_t out)
+{
+    switch (out) {
+    case GEMM_F16: return gemm_relu_tc_kernel<PAIR, BMN, __half>;
+    case GEMM_BF16: return gemm_relu_tc_kernel<PAIR, BMN, __nv_bfloat16>;
+    default: return gemm_relu_tc_kernel<PAIR, BMN, float>;
+    }
+}
+
+GemmKernelFn pick_kernel(bool pair, bool b_mn, gemm_dtype_t out)
+{
+    if (pair) return b_mn ? pick_out<true, true>(out) : pick_out<true, false>(out);
+    return b_mn ? pick_out<false, true>(out) : pick_out<false, false>(out);
+}
+
+int variant_index(bool pair, bool b_mn, gemm_dtype_t out)
+{
+    return (pair ? 6 : 0) + (b_mn ? 3 : 0) + static_cast<int>(out);
+}
+
+// ------------------------------------------------------------------ devices
+struct DeviceInfo {
+    bool ready = false;
+    bool ok = false;
+    int sms = 0;
+    int max_pair_clusters = 0;
+    bool attr_set[12] = {};
+};
+
+std::mutex g_dev_mutex;
+DeviceInfo g_dev[kMaxDevices];
+
+gemm_status_t ensure_kernel_attr(DeviceInfo &d, bool pair, bool b_mn, gemm_dtype_t out)
+{
+    const int v = variant_index(pair, b_mn, out);
+    if (d.attr_set[v]) return GEMM_OK;
+    const int smem = pair ? TileCfg<true>::kSmemBytes : TileCfg<false>::kSmemBytes;
+    cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void *>(pick_kernel(pair, b_mn, out)),
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    d.attr_set[v] = true;
+    return GEMM_OK;
+}
+
+gemm_status_t device_info(DeviceInfo **out)
+{
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        t_last_cuda_error = std::string("cudaGetDevice: ") + cudaGetErrorString(e);
+        return GEMM_ERR_NO_DEVICE;
+    }
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    DeviceInfo &d = g_dev[dev];
+    if (!d.ready) {
+        int major = 0, minor = 0, sms = 0;
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        d.ready = true;
+        d.ok = (major == 10 && minor == 0 && sms > 0);
+        d.sms = sms;
+        if (d.ok) {
+            // how many 2-CTA clusters of the pair kernel fit at once
+            gemm_status_t st = ensure_kernel_attr(d, true, false, GEMM_F16);
+            if (st != GEMM_OK) return st;
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(2 * sms, 1, 1);
+            cfg.blockDim = dim3(kThreads, 1, 1);
+            cfg.dynamicSmemBytes = TileCfg<true>::kSmemBytes;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 2;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int clusters = 0;
+            e = cudaOccupancyMaxActiveClusters(
+                &clusters, reinterpret_cast<const void *>(pick_kernel(true, false, GEMM_F16)), &cfg);
+            if (e != cudaSuccess || clusters <= 0) clusters = sms / 2;
+            d.max_pair_clusters = std::min(clusters, sms / 2);
+        }
+    }
+    if (!d.ok) {
+        t_last_cuda_error = "device is not compute capability 10.0 (sm_100a build)";
+        return GEMM_ERR_NO_DEVICE;
+    }
+    *out = &d;
+    return GEMM_OK;
+}
+
+// ------------------------------------------------------------------ plan
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
+
+size_t dtype_size(gemm_dtype_t t) { return t == GEMM_F32 ? 4 : 2; }
+
+struct Layout {
+    // byte offsets inside the workspace
+    int64_t a_off = 0, b_off = 0, split_off = 0, total = 0;
+    int64_t a_pitch = 0, b_pitch = 0;  // elements
+};
+
+bool misaligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+
+gemm_status_t make_plan(int64_t M, int64_t N, int64_t K, gemm_dtype_t in, gemm_dtype_t out,
+                        int trans_b, const void *A, const void *B, int num_sms,
+                        int max_pair_clusters, const gemm_relu_options_t *opts,
+                        gemm_relu_plan_t *plan, Layout *lay)
+{
+    if (M < 0 || N < 0 || K < 0 || num_sms <= 0) return GEMM_ERR_INVALID_ARG;
+    if (in != GEMM_F16 && in != GEMM_BF16) return GEMM_ERR_UNSUPPORTED_DTYPE;
+    if (out != GEMM_F16 && out != GEMM_BF16 && out != GEMM_F32) return GEMM_ERR_UNSUPPORTED_DTYPE;
+    // the kernels index rows/columns with 32-bit ints; TMA dims must be < 2^32
+    if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX - kBK) return GEMM_ERR_INVALID_ARG;
+    gemm_relu_options_t o = {};
+    if (opts) o = *opts;
+    if (o.cta_pair < 0 || o.cta_pair > 2 || o.split_k < 0 || o.panel < 0 || o.max_ctas < 0)
+        return GEMM_ERR_INVALID_ARG;
+
+    gemm_relu_plan_t p = {};
+    p.tile_n = kBN;
+    p.tile_k = kBK;
+    p.kblocks = static_cast<int>(ceil_div(K, kBK));
+    const int64_t tiles_n = ceil_div(N, kBN);
+    const int64_t tiles1 = ceil_div(M, kBM) * tiles_n;  // 1-CTA tiling
+
+    int64_t split = o.split_k;
+    if (split == 0) {
+        split = 1;
+        // too few output tiles to occupy the SMs: split K, keeping >= 4 K blocks each
+        if (tiles1 > 0 && tiles1 * 2 <= num_sms && p.kblocks >= 8) {
+            split = std::max<int64_t>(1, num_sms / tiles1);
+            split = std::min<int64_t>(split, p.kblocks / 4);
+            split = std::min<int64_t>(split, 32);
+        }
+    }
+    if (p.kblocks > 0) split = std::max<int64_t>(1, std::min<int64_t>(split, p.kblocks));
+    else split = 1;
+
+    bool pair;
+    if (split > 1) pair = false;
+    else if (o.cta_pair == GEMM_CTA_PAIR) pair = true;
+    else if (o.cta_pair == GEMM_CTA_SINGLE) pair = false;
+    else pair = M > kBM;
+
+    p.cta_pair = pair ? 1 : 0;
+    p.tile_m = pair ? 2 * kBM : kBM;
+    const int64_t tiles_m = ceil_div(M, p.tile_m);
+    const int64_t units = tiles_m * tiles_n * split;
+    if (units > INT32_MAX) return GEMM_ERR_INVALID_ARG;
+    p.tiles_m = static_cast<int>(tiles_m);
+    p.tiles_n = static_cast<int>(tiles_n);
+    p.split_k = static_cast<int>(split);
+    p.panel = o.panel > 0 ? o.panel : kDefaultPanel;
+    if (p.tiles_m > 0) p.panel = std::min(p.panel, p.tiles_m);
+    p.units = static_cast<int>(units);
+    p.stages = pair ? TileCfg<true>::kStages : TileCfg<false>::kStages;
+
+    int64_t grid;
+    if (pair) {
+        int64_t clusters = max_pair_clusters > 0 ? max_pair_clusters : num_sms / 2;
+        if (o.max_ctas > 0) clusters = std::min<int64_t>(clusters, std::max(1, o.max_ctas / 2));
+        grid = 2 * std::min<int64_t>(units, std::max<int64_t>(1, clusters));
+    } else {
+        int64_t ctas = num_sms;
+        if (o.max_ctas > 0) ctas = std::min<int64_t>(ctas, o.max_ctas);
+        grid = std::min<int64_t>(units, ctas);
+    }
+    p.grid_ctas = static_cast<int>(grid);
+
+    // TMA reads rows whose byte pitch and base address are 16-byte aligned
+    const int64_t a_row_bytes = K * 2;
+    const int64_t b_row_bytes = (trans_b ? K : N) * 2;
+    p.pack_a = (o.force_pack || misaligned16(A) || (a_row_bytes % 16) != 0) ? 1 : 0;
+    p.pack_b = (o.force_pack || misaligned16(B) || (b_row_bytes % 16) != 0) ? 1 : 0;
+    if (K == 0 || M == 0 || N == 0) p.pack_a = p.pack_b = 0;
+
+    Layout l;
+    int64_t off = 0;
+    if (p.pack_a) {
+        l.a_pitch = round_up(K, 8);
+        l.a_off = off;
+        off = round_up(off + M * l.a_pitch * 2, 256);
+    }
+    if (p.pack_b) {
+        const int64_t rows = trans_b ? N : K, cols = trans_b ? K : N;
+        l.b_pitch = round_up(cols, 8);
+        l.b_off = off;
+        off = round_up(off + rows * l.b_pitch * 2, 256);
+    }
+    if (p.split_k > 1) {
+        l.split_off = off;
+        off = round_up(off + static_cast<int64_t>(p.split_k) * M * N * 4, 256);
+    }
+    l.total = off;
+    p.workspace_bytes = off;
+    if (plan) *plan = p;
+    if (lay) *lay = l;
+    return GEMM_OK;
+}
+
+// ------------------------------------------------------------------ workspace
+struct Workspace {
+    void *ptr = nullptr;
+    int64_t bytes = 0;
+};
+std::mutex g_ws_mutex;
+std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
+
+gemm_status_t get_workspace(cudaStream_t stream, int64_t bytes, void **out)
+{
+    *out = nullptr;
+    if (bytes <= 0) return GEMM_OK;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lock(g_ws_mutex);
+    Workspace &w = g_ws[{dev, stream}];
+    if (w.bytes < bytes) {
+        if (w.ptr) {
+            cudaError_t e = cudaStreamSynchronize(stream);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+            cudaFree(w.ptr);
+            w.ptr = nullptr;
+            w.bytes = 0;
+        }
+        const int64_t want = round_up(bytes + bytes / 4, 1 << 20);
+        cudaError_t e = cudaMalloc(&w.ptr, static_cast<size_t>(want));
+        if (e != cudaSuccess) {
+            w.ptr = nullptr;
+            return cuda_fail(e, "cudaMalloc(workspace)");
+        }
+        w.bytes = want;
+    }
+    *out = w.ptr;
+    return GEMM_OK;
+}
+
+// ------------------------------------------------------------------ tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D map over a row-major 16-bit matrix: inner extent `inner` (contiguous),
+// `outer` rows `pitch_elems` apart, box {box_inner, box_outer}, 128-byte swizzle,
+// out-of-range elements read as zero.
+gemm_status_t encode_2d(CUtensorMap *map, const void *base, gemm_dtype_t dt, int64_t inner,
+                        int64_t outer, int64_t pitch_elems, int box_inner, int box_outer)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) {
+        t_last_cuda_error = "cuTensorMapEncodeTiled entry point not available";
+        return GEMM_ERR_CUDA;
+    }
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(pitch_elems * 2)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_outer)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, dt == GEMM_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                    2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        t_last_cuda_error = "cuTensorMapEncodeTiled failed with CUresult " + std::to_string(static_cast<int>(r));
+        return GEMM_ERR_CUDA;
+    }
+    return GEMM_OK;
+}
+
+// tcgen05 instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A/B type
+// (bits 7-9 / 10-12: 0 fp16, 1 bf16), A K-major (bit 15 = 0), B major (bit
+// 16: 0 K-major, 1 MN-major), N >> 3 (bits 17-22), M >> 4 (bits 24-28).
+uint32_t make_idesc(gemm_dtype_t in, bool b_mn, int mma_m, int mma_n)
+{
+    const uint32_t t = in == GEMM_BF16 ? 1u : 0u;
+    return (1u << 4) | (t << 7) | (t << 10) | ((b_mn ? 1u : 0u) << 16) |
+           (static_cast<uint32_t>(mma_n >> 3) << 17) | (static_cast<uint32_t>(mma_m >> 4) << 24);
+}
+
+gemm_status_t launch_repitch(const void *src, int64_t rows, int64_t cols, void *dst,
+                             int64_t pitch, cudaStream_t stream)
+{
+    dim3 block(256);
+    dim3 grid(static_cast<unsigned>(std::min<int64_t>(ceil_div(cols, 256), 64)),
+              static_cast<unsigned>(std::min<int64_t>(rows, 65535)));
+    repitch_kernel<<<grid, block, 0, stream>>>(static_cast<const uint16_t *>(src), rows, cols,
+                                                static_cast<uint16_t *>(dst), pitch);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? GEMM_OK : cuda_fail(e, "repitch launch");
+}
+
+template <typename OutT>
+void launch_reduce_t(const float *ws, void *C, int64_t n_total, int splits, int64_t split_stride,
+                     int relu, int vec4, int grid, cudaStream_t stream)
+{
+    splitk_reduce_kernel<OutT><<<grid, 256, 0, stream>>>(ws, static_cast<OutT *>(C), n_total,
+                                                          splits, split_stride, relu, vec4);
+}
+
+gemm_status_t run(const void *A, const void *B, void *C, int64_t M, int64_t N, int64_t K,
+                  gemm_dtype_t in, gemm_dtype_t out, int trans_b, int relu, void *stream_v,
+                  const gemm_relu_options_t *opts)
+{
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+    gemm_relu_plan_t plan;
+    Layout lay;
+    // argument checks first (no device needed)
+    gemm_status_t st = make_plan(M, N, K, in, out, trans_b, A, B, 148, 74, opts, &plan, &lay);
+    if (st != GEMM_OK) return st;
+    if (M == 0 || N == 0) return GEMM_OK;
+    if (!C || (K > 0 && (!A || !B))) return GEMM_ERR_INVALID_ARG;
+
+    DeviceInfo *dev = nullptr;
+    st = device_info(&dev);
+    if (st != GEMM_OK) return st;
+    st = make_plan(M, N, K, in, out, trans_b, A, B, dev->sms, dev->max_pair_clusters, opts, &plan,
+                   &lay);
+    if (st != GEMM_OK) return st;
+
+    const size_t osz = dtype_size(out);
+    if (K == 0) {  // empty sum: relu(0) = 0
+        cudaError_t e = cudaMemsetAsync(C, 0, static_cast<size_t>(M * N) * osz, stream);
+        return e == cudaSuccess ? GEMM_OK : cuda_fail(e, "cudaMemsetAsync");
+    }
+
+    void *ws = nullptr;
+    st = get_workspace(stream, lay.total, &ws);
+    if (st != GEMM_OK) return st;
+    char *wsb = static_cast<char *>(ws);
+
+    const void *a_src = A;
+    int64_t a_pitch = K;
+    if (plan.pack_a) {
+        st = launch_repitch(A, M, K, wsb + lay.a_off, lay.a_pitch, stream);
+        if (st != GEMM_OK) return st;
+        a_src = wsb + lay.a_off;
+        a_pitch = lay.a_pitch;
+    }
+    const void *b_src = B;
+    int64_t b_pitch = trans_b ? K : N;
+    if (plan.pack_b) {
+        st = launch_repitch(B, trans_b ? N : K, trans_b ? K : N, wsb + lay.b_off, lay.b_pitch, stream);
+        if (st != GEMM_OK) return st;
+        b_src = wsb + lay.b_off;
+        b_pitch = lay.b_pitch;
+    }
+
+    const bool pair = plan.cta_pair != 0;
+    const bool b_mn = !trans_b;
+    const int bn_cta = pair ? kBN / 2 : kBN;
+    CUtensorMap tmA, tmB;
+    st = encode_2d(&tmA, a_src, in, K, M, a_pitch, kBK, kBM);
+    if (st != GEMM_OK) return st;
+    if (b_mn)
+        st = encode_2d(&tmB, b_src, in, N, K, b_pitch, 64, kBK);
+    else
+        st = encode_2d(&tmB, b_src, in, K, N, b_pitch, kBK, bn_cta);
+    if (st != GEMM_OK) return st;
+
+    const bool split = plan.split_k > 1;
+    const gemm_dtype_t kout = split ? GEMM_F32 : out;
+    GemmParams p = {};
+    p.C = split ? static_cast<void *>(wsb + lay.split_off) : C;
+    p.ldc = N;
+    p.split_stride = split ? M * N : 0;
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(N);
+    p.K = static_cast<int>(K);
+    p.tiles_m = plan.tiles_m;
+    p.tiles_n = plan.tiles_n;
+    p.splits = plan.split_k;
+    p.kblocks = plan.kblocks;
+    p.panel = plan.panel;
+    p.num_units = plan.units;
+    p.relu = split ? 0 : (relu ? 1 : 0);
+    p.vec_ok = (!misaligned16(p.C) && ((N * static_cast<int64_t>(dtype_size(kout))) % 16) == 0) ? 1 : 0;
+    p.idesc = make_idesc(in, b_mn, pair ? 2 * kBM : kBM, kBN);
+    p.timeout_ns = (opts && opts->timeout_ns) ? opts->timeout_ns : kDefaultTimeoutNs;
+
+    {
+        std::lock_guard<std::mutex> lock(g_dev_mutex);
+        st = ensure_kernel_attr(*dev, pair, b_mn, kout);
+    }
+    if (st != GEMM_OK) return st;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(plan.grid_ctas), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = pair ? TileCfg<true>::kSmemBytes : TileCfg<false>::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = pair ? 2 : 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pair ? 1 : 0;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, pick_kernel(pair, b_mn, kout), tmA, tmB, p);
+    if (e != cudaSuccess) return cuda_fail(e, "gemm kernel launch");
+
+    if (split) {
+        const int64_t n_total = M * N;
+        const int vec4 = ((n_total % 4) == 0 && !misaligned16(C) && (osz * 4) % 4 == 0) ? 1 : 0;
+        const int grid = static_cast<int>(std::min<int64_t>(ceil_div(n_total / (vec4 ? 4 : 1), 256),
+                                                            static_cast<int64_t>(dev->sms) * 8));
+        const float *wsf = reinterpret_cast<const float *>(wsb + lay.split_off);
+        switch (out) {
+        case GEMM_F16: launch_reduce_t<__half>(wsf, C, n_total, plan.split_k, M * N, relu ? 1 : 0, vec4, grid, stream); break;
+        case GEMM_BF16: launch_reduce_t<__nv_bfloat16>(wsf, C, n_total, plan.split_k, M * N, relu ? 1 : 0, vec4, grid, stream); break;
+        default: launch_reduce_t<float>(wsf, C, n_total, plan.split_k, M * N, relu ? 1 : 0, vec4, grid, stream); break;
+        }
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "split-K reduce launch");
+    }
+    return GEMM_OK;
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+gemm_status_t gemm_relu(const void *A, const void *B, void *C, int64_t M, int64_t N, int64_t K,
+                        gemm_dtype_t in_dtype, gemm_dtype_t out_dtype, int trans_b, int relu,
+                        void *stream)
+{
+    return run(A, B, C, M, N, K, in_dtype, out_dtype, trans_b, relu, stream, nullptr);
+}
+
+gemm_status_t gemm_relu_ex(const void *A, const void *B, void *C, int64_t M, int64_t N,
+                           int64_t K, gemm_dtype_t in_dtype, gemm_dtype_t out_dtype, int trans_b,
+                           int relu, void *stream, const gemm_relu_options_t *opts)
+{
+    return run(A, B, C, M, N, K, in_dtype, out_dtype, trans_b, relu, stream, opts);
+}
+
+gemm_status_t gemm_relu_plan(int64_t M, int64_t N, int64_t K, gemm_dtype_t in_dtype,
+                             gemm_dtype_t out_dtype, int trans_b, const void *A, const void *B,
+                             int num_sms, int max_pair_clusters, const gemm_relu_options_t *opts,
+                             gemm_relu_plan_t *plan)
+{
+    if (!plan) return GEMM_ERR_INVALID_ARG;
+    return make_plan(M, N, K, in_dtype, out_dtype, trans_b, A, B, num_sms, max_pair_clusters, opts,
+                     plan, nullptr);
+}
+
+gemm_status_t gemm_relu_plan_unit(const gemm_relu_plan_t *plan, int u, gemm_relu_unit_t *unit)
+{
+    if (!plan || !unit || u < 0 || u >= plan->units || plan->split_k < 1 || plan->panel < 1)
+        return GEMM_ERR_INVALID_ARG;
+    const WorkUnit w = decode_unit(u, plan->tiles_m, plan->tiles_n, plan->split_k, plan->kblocks,
+                                   plan->panel);
+    unit->tile_row = w.m_tile;
+    unit->tile_col = w.n_tile;
+    unit->kb_begin = w.kb0;
+    unit->kb_end = w.kb1;
+    unit->split = w.split;
+    return GEMM_OK;
+}
+
+const char *gemm_relu_status_string(gemm_status_t s)
+{
+    switch (s) {
+    case GEMM_OK: return "ok";
+    case GEMM_ERR_INVALID_ARG: return "invalid argument";
+    case GEMM_ERR_UNSUPPORTED_DTYPE: return "unsupported dtype";
+    case GEMM_ERR_MISALIGNED: return "misaligned operand";
+    case GEMM_ERR_CUDA: return "CUDA error";
+    case GEMM_ERR_TIMEOUT: return "device wait timed out";
+    case GEMM_ERR_NO_DEVICE: return "no compute capability 10.0 device";
+    }
+    return "unknown status";
+}
+
+const char *gemm_relu_last_cuda_error(void) { return t_last_cuda_error.c_str(); }
+
+gemm_status_t gemm_relu_last_device_error(uint32_t *detail)
+{
+    DeviceInfo *dev = nullptr;
+    gemm_status_t st = device_info(&dev);
+    if (st != GEMM_OK) return st;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    uint32_t v = 0, zero = 0;
+    e = cudaMemcpyFromSymbol(&v, g_gemm_device_error, sizeof(v));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyFromSymbol");
+    e = cudaMemcpyToSymbol(g_gemm_device_error, &zero, sizeof(zero));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyToSymbol");
+    if (detail) *detail = v;
+    return v ? GEMM_ERR_TIMEOUT : GEMM_OK;
+}
+
+gemm_status_t gemm_relu_selftest_timeout(uint64_t timeout_ns, void *stream_v)
+{
+    DeviceInfo *dev = nullptr;
+    gemm_status_t st = device_info(&dev);
+    if (st != GEMM_OK) return st;
+    if (timeout_ns == 0 || timeout_ns > 10000000000ull) return GEMM_ERR_INVALID_ARG;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+    int *d_out = nullptr;
+    cudaError_t e = cudaMalloc(&d_out, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc");
+    int h_out = -1;
+    selftest_timeout_kernel<<<1, 32, 0, stream>>>(timeout_ns, d_out);
+    e = cudaGetLastError();
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e == cudaSuccess) e = cudaMemcpy(&h_out, d_out, sizeof(int), cudaMemcpyDeviceToHost);
+    cudaFree(d_out);
+    if (e != cudaSuccess) return cuda_fail(e, "self-test");
+    return h_out == 0 ? GEMM_ERR_TIMEOUT : GEMM_OK;
+}
+
+gemm_status_t gemm_relu_release_workspace(void)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GEMM_ERR_NO_DEVICE;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    std::lock_guard<std::mutex> lock(g_ws_mutex);
+    for (auto it = g_ws.begin(); it != g_ws.end();) {
+        if (it->first.first == dev) {
+            cudaFree(it->second.ptr);
+            it = g_ws.erase(it);
+        } else {
+            ++it;
+        }
+    }
+    return GEMM_OK;
+}
+
+int gemm_relu_version(void) { return kVersion; }
+
+}  // extern "C"
