@@ -169,6 +169,43 @@ GEMM_RELU_API gemm_status_t gemm_relu_release_workspace(void);
 /* Library version: major * 10000 + minor * 100 + patch. */
 GEMM_RELU_API int gemm_relu_version(void);
 
+/* ---- Split-K GEMM + ReLU that allocates no device memory -------------------
+ * (No counterpart in the paper; it exists for callers, not for the method.)
+ *
+ * Some callers cannot call cudaMalloc while they run: code inside a memory
+ * pool or arena that owns all device memory, a process that must not grow
+ * its footprint after start-up, or a caller holding a lock under which the
+ * implicit device synchronisation of a first cudaMalloc/cudaFree is not
+ * allowed.  gemm_relu may allocate (it grows a per-stream workspace on
+ * demand); this entry point never does.  It runs the split-K path (1-CTA
+ * kernel writing fp32 partial sums, then the fixed-order reduction with the
+ * ReLU and the cast) with its partial sums in a static device array of
+ * GEMM_RELU_NOALLOC_SCRATCH_BYTES (16 MiB) that the library holds on every
+ * GPU that loads it, until the process exits.
+ *
+ * Arguments are those of gemm_relu plus split_k (0 = the automatic choice,
+ * >= 1 = that many K splits, clamped to ceil(K / 64)).  The caller still
+ * owns and passes A, B and C (device pointers).  Returns
+ *   GEMM_ERR_INVALID_ARG   if split_k * M * N * 4 bytes of partial sums would
+ *                          not fit in GEMM_RELU_NOALLOC_SCRATCH_BYTES (or on
+ *                          the usual argument errors);
+ *   GEMM_ERR_MISALIGNED    if A or B has a base address or row pitch that is
+ *                          not a multiple of 16 bytes (re-pitching them would
+ *                          need memory; gemm_relu accepts such operands).
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  All calls share the one array and it keeps
+ * the last call's partial sums; every call overwrites every partial it later
+ * reads, so nothing has to start at zero.  Calls whose executions overlap on
+ * the GPU (for example on two streams at once) race on the array: serialise
+ * them. */
+#define GEMM_RELU_NOALLOC_SCRATCH_BYTES (16ll * 1024 * 1024)
+GEMM_RELU_API gemm_status_t gemm_relu_splitk_noalloc(const void *A, const void *B, void *C,
+                                                     int64_t M, int64_t N, int64_t K,
+                                                     gemm_dtype_t in_dtype, gemm_dtype_t out_dtype,
+                                                     int trans_b, int relu, int split_k,
+                                                     void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -20,6 +20,7 @@ from ._abi import (  # noqa: F401
     GEMM_F32,
     GEMM_OK,
     LIB_PATH,
+    NOALLOC_SCRATCH_BYTES,
     GemmError,
     GemmOptions,
     gemm_relu,
@@ -30,6 +31,7 @@ from ._abi import (  # noqa: F401
     gemm_relu_plan_unit,
     gemm_relu_release_workspace,
     gemm_relu_selftest_timeout,
+    gemm_relu_splitk_noalloc,
     gemm_relu_status_string,
     gemm_relu_version,
     load,

@@ -35,7 +35,11 @@ EXPORTS = (
     "gemm_relu", "gemm_relu_ex", "gemm_relu_plan", "gemm_relu_status_string",
     "gemm_relu_last_cuda_error", "gemm_relu_last_device_error", "gemm_relu_selftest_timeout",
     "gemm_relu_release_workspace", "gemm_relu_version", "gemm_relu_plan_unit",
+    "gemm_relu_splitk_noalloc",
 )
+
+# size of the static device array behind gemm_relu_splitk_noalloc (header constant)
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 _DTYPE_CODE = {torch.float16: GEMM_F16, torch.bfloat16: GEMM_BF16, torch.float32: GEMM_F32}
 
@@ -89,6 +93,7 @@ def load():
             gemm_args = [vp, vp, vp, i64, i64, i64, i32, i32, i32, i32, vp]
             lib.gemm_relu.argtypes = gemm_args
             lib.gemm_relu_ex.argtypes = gemm_args + [ctypes.POINTER(GemmOptions)]
+            lib.gemm_relu_splitk_noalloc.argtypes = gemm_args[:10] + [i32, vp]
             lib.gemm_relu_plan.argtypes = [i64, i64, i64, i32, i32, i32, vp, vp, i32, i32,
                                            ctypes.POINTER(GemmOptions), ctypes.POINTER(GemmPlan)]
             lib.gemm_relu_plan_unit.argtypes = [ctypes.POINTER(GemmPlan), i32,
@@ -103,7 +108,7 @@ def load():
             lib.gemm_relu_version.argtypes = []
             for name in ("gemm_relu", "gemm_relu_ex", "gemm_relu_plan", "gemm_relu_last_device_error",
                          "gemm_relu_selftest_timeout", "gemm_relu_release_workspace",
-                         "gemm_relu_version", "gemm_relu_plan_unit"):
+                         "gemm_relu_version", "gemm_relu_plan_unit", "gemm_relu_splitk_noalloc"):
                 getattr(lib, name).restype = i32
             _lib = lib
     return _lib
@@ -171,6 +176,16 @@ def gemm_relu_ex(A, B, C, M, N, K, in_dtype, out_dtype, trans_b, relu, stream=No
     st = load().gemm_relu_ex(_ptr(A), _ptr(B), _ptr(C), int(M), int(N), int(K), _dtype(in_dtype),
                              _dtype(out_dtype), int(bool(trans_b)), int(bool(relu)),
                              _stream(stream), ctypes.byref(o) if o is not None else None)
+    return _check(st) if check else st
+
+
+def gemm_relu_splitk_noalloc(A, B, C, M, N, K, in_dtype, out_dtype, trans_b, relu, split_k=0,
+                             stream=None, check: bool = True) -> int:
+    """Split-K GEMM + ReLU whose partial sums live in the library's static device
+    array: the call allocates no device memory (for callers that cannot)."""
+    st = load().gemm_relu_splitk_noalloc(_ptr(A), _ptr(B), _ptr(C), int(M), int(N), int(K),
+                                         _dtype(in_dtype), _dtype(out_dtype), int(bool(trans_b)),
+                                         int(bool(relu)), int(split_k), _stream(stream))
     return _check(st) if check else st
 
 

@@ -588,3 +588,134 @@ gemm_status_t gemm_relu_release_workspace(void)
 int gemm_relu_version(void) { return kVersion; }
 
 }  // extern "C"
+
+// ====================================================================== no-alloc split-K
+// The split-K path of gemm_relu with its fp32 partial sums in a static device
+// array instead of the per-stream workspace, for callers that must not
+// allocate device memory (see the header).  It reuses the 1-CTA kernel and
+// the reduction kernel unchanged.
+namespace {
+
+constexpr int64_t kNoAllocScratchBytes = GEMM_RELU_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+std::mutex g_noalloc_mutex;
+void *g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (host code cannot use the symbol itself as an address).
+gemm_status_t noalloc_scratch(void **out)
+{
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GEMM_ERR_NO_DEVICE;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess || !p) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return GEMM_OK;
+}
+
+}  // namespace
+
+extern "C" gemm_status_t gemm_relu_splitk_noalloc(const void *A, const void *B, void *C,
+                                                  int64_t M, int64_t N, int64_t K,
+                                                  gemm_dtype_t in, gemm_dtype_t out, int trans_b,
+                                                  int relu, int split_k, void *stream_v)
+{
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+    if (split_k < 0) return GEMM_ERR_INVALID_ARG;
+    gemm_relu_options_t o = {};
+    o.cta_pair = GEMM_CTA_SINGLE;
+    o.split_k = split_k;
+    gemm_relu_plan_t plan;
+    Layout lay;
+    gemm_status_t st = make_plan(M, N, K, in, out, trans_b, A, B, 148, 74, &o, &plan, &lay);
+    if (st != GEMM_OK) return st;
+    if (M == 0 || N == 0) return GEMM_OK;
+    if (!C || (K > 0 && (!A || !B))) return GEMM_ERR_INVALID_ARG;
+
+    DeviceInfo *dev = nullptr;
+    st = device_info(&dev);
+    if (st != GEMM_OK) return st;
+    st = make_plan(M, N, K, in, out, trans_b, A, B, dev->sms, dev->max_pair_clusters, &o, &plan,
+                   &lay);
+    if (st != GEMM_OK) return st;
+    if (plan.pack_a || plan.pack_b) return GEMM_ERR_MISALIGNED;
+    const size_t osz = dtype_size(out);
+    if (K == 0) {
+        cudaError_t e = cudaMemsetAsync(C, 0, static_cast<size_t>(M * N) * osz, stream);
+        return e == cudaSuccess ? GEMM_OK : cuda_fail(e, "cudaMemsetAsync");
+    }
+    const bool split = plan.split_k > 1;
+    const int64_t partial_bytes = split ? static_cast<int64_t>(plan.split_k) * M * N * 4 : 0;
+    if (partial_bytes > kNoAllocScratchBytes) return GEMM_ERR_INVALID_ARG;
+
+    void *scratch = nullptr;
+    if (split) {
+        st = noalloc_scratch(&scratch);
+        if (st != GEMM_OK) return st;
+    }
+
+    const bool b_mn = !trans_b;
+    CUtensorMap tmA, tmB;
+    st = encode_2d(&tmA, A, in, K, M, K, kBK, kBM);
+    if (st != GEMM_OK) return st;
+    if (b_mn)
+        st = encode_2d(&tmB, B, in, N, K, N, 64, kBK);
+    else
+        st = encode_2d(&tmB, B, in, K, N, K, kBK, kBN);
+    if (st != GEMM_OK) return st;
+
+    const gemm_dtype_t kout = split ? GEMM_F32 : out;
+    GemmParams p = {};
+    p.C = split ? scratch : C;
+    p.ldc = N;
+    p.split_stride = split ? M * N : 0;
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(N);
+    p.K = static_cast<int>(K);
+    p.tiles_m = plan.tiles_m;
+    p.tiles_n = plan.tiles_n;
+    p.splits = plan.split_k;
+    p.kblocks = plan.kblocks;
+    p.panel = plan.panel;
+    p.num_units = plan.units;
+    p.relu = split ? 0 : (relu ? 1 : 0);
+    p.vec_ok = (!misaligned16(p.C) && ((N * static_cast<int64_t>(dtype_size(kout))) % 16) == 0) ? 1 : 0;
+    p.idesc = make_idesc(in, b_mn, kBM, kBN);
+    p.timeout_ns = kDefaultTimeoutNs;
+    {
+        std::lock_guard<std::mutex> lock(g_dev_mutex);
+        st = ensure_kernel_attr(*dev, false, b_mn, kout);
+    }
+    if (st != GEMM_OK) return st;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(plan.grid_ctas), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = TileCfg<false>::kSmemBytes;
+    cfg.stream = stream;
+    cfg.numAttrs = 0;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, pick_kernel(false, b_mn, kout), tmA, tmB, p);
+    if (e != cudaSuccess) return cuda_fail(e, "no-alloc gemm kernel launch");
+    if (split) {
+        const int64_t n_total = M * N;
+        const int vec4 = (n_total % 4) == 0 ? 1 : 0;
+        const int grid = static_cast<int>(std::min<int64_t>(ceil_div(n_total / (vec4 ? 4 : 1), 256),
+                                                            static_cast<int64_t>(dev->sms) * 8));
+        const float *wsf = static_cast<const float *>(scratch);
+        switch (out) {
+        case GEMM_F16: launch_reduce_t<__half>(wsf, C, n_total, plan.split_k, M * N, relu ? 1 : 0, vec4, grid, stream); break;
+        case GEMM_BF16: launch_reduce_t<__nv_bfloat16>(wsf, C, n_total, plan.split_k, M * N, relu ? 1 : 0, vec4, grid, stream); break;
+        default: launch_reduce_t<float>(wsf, C, n_total, plan.split_k, M * N, relu ? 1 : 0, vec4, grid, stream); break;
+        }
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "no-alloc split-K reduce launch");
+    }
+    return GEMM_OK;
+}
