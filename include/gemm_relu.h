@@ -82,6 +82,8 @@ typedef struct {
     int force_pack;      /* 1 = copy A and B through the 16-byte-pitched workspace        */
     int max_ctas;        /* 0 = one CTA per SM; >= 1 caps the persistent grid (CTAs)      */
     uint64_t timeout_ns; /* 0 = 1 s; bound on every in-kernel barrier wait                */
+    int stage_k;         /* 0 = auto (128 for the CTA pair, 64 otherwise); 64 or 128: K per
+                            shared-memory pipeline stage of the CTA-pair kernel            */
 } gemm_relu_options_t;
 /* cta_pair: 0 = auto, 1 = force the 2-CTA (256 x 256 tile, cta_group::2)
  * kernel, 2 = force the 1-CTA (128 x 256 tile) kernel.  Split-K always uses

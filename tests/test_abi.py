@@ -62,6 +62,7 @@ def plan(w: wl.Workload, **opt):
 def test_plans_for_the_workloads(lib):
     p = plan(wl.WORKLOADS["square8192_f16"])
     assert (p["cta_pair"], p["tile_m"], p["tile_n"], p["split_k"]) == (1, 256, 256, 1)
+    assert (p["tile_k"], p["kblocks"], p["stages"]) == (128, 64, 3)
     assert (p["tiles_m"], p["tiles_n"], p["units"], p["grid_ctas"]) == (32, 32, 1024, 148)
     assert p["pack_a"] == p["pack_b"] == 0 and p["workspace_bytes"] == 0
 
@@ -70,7 +71,7 @@ def test_plans_for_the_workloads(lib):
 
     p = plan(wl.WORKLOADS["tail5000x3001x2050_f16"])
     assert p["pack_a"] == 1 and p["pack_b"] == 1          # 4100- and 6002-byte row pitches
-    assert p["kblocks"] == 33 and p["tiles_m"] == 20 and p["tiles_n"] == 12
+    assert p["kblocks"] == 17 and p["tiles_m"] == 20 and p["tiles_n"] == 12   # K tail 2050 % 128
 
     p = plan(wl.WORKLOADS["skinny64x8192x8192_f16"])
     assert p["cta_pair"] == 0 and p["split_k"] == 4 and p["units"] == 128
@@ -94,6 +95,11 @@ def test_options_override_the_plan(lib):
     assert plan(w, max_ctas=10, cta_pair=g.GEMM_CTA_PAIR)["grid_ctas"] == 10
     assert plan(w, force_pack=1)["pack_a"] == 1
     assert plan(w, panel=3)["panel"] == 3
+    p = plan(w, stage_k=64)
+    assert (p["tile_k"], p["kblocks"], p["stages"]) == (64, 64, 7)
+    assert plan(w, cta_pair=g.GEMM_CTA_SINGLE, stage_k=128)["tile_k"] == 64   # 1-CTA: 64 only
+    with pytest.raises(g.GemmError):
+        plan(w, stage_k=96)
 
 
 def test_misaligned_base_pointer_is_repitched(lib):
@@ -110,6 +116,7 @@ def test_misaligned_base_pointer_is_repitched(lib):
     (300, 700, 1000, {"split_k": 7, "panel": 3}),
     (1000, 300, 130, {"cta_pair": g.GEMM_CTA_SINGLE, "panel": 5}),
     (257, 257, 65, {"panel": 1}),
+    (600, 300, 1000, {"stage_k": 64}),
 ])
 def test_units_cover_every_tile_and_k_block_once(lib, M, N, K, opt):
     p = g.gemm_relu_plan(M, N, K, torch.float16, torch.float16, False, options=opt or None)

@@ -94,6 +94,7 @@ VARIANTS = {
     "auto": None,
     "single": {"cta_pair": g.GEMM_CTA_SINGLE},
     "pair": {"cta_pair": g.GEMM_CTA_PAIR},
+    "pair_k64": {"cta_pair": g.GEMM_CTA_PAIR, "stage_k": 64},
     "split3": {"split_k": 3},
     "packed": {"force_pack": 1},
     "few_ctas": {"max_ctas": 3, "panel": 2},
@@ -111,7 +112,7 @@ def test_shapes_fp16(M, N, K, trans_b, variant):
 @pytest.mark.parametrize("in_dtype", [F16, BF16])
 @pytest.mark.parametrize("trans_b", [False, True])
 @pytest.mark.parametrize("relu", [True, False])
-@pytest.mark.parametrize("variant", ["auto", "single", "split3"])
+@pytest.mark.parametrize("variant", ["auto", "single", "split3", "pair_k64"])
 def test_dtypes_and_relu(in_dtype, out_dtype, trans_b, relu, variant):
     full_case(300, 520, 330, in_dtype, out_dtype, trans_b, relu, VARIANTS[variant], seed=7,
               dist="normal")
@@ -158,7 +159,7 @@ def test_full_size_workloads_sampled(name):
 
 
 # ---------------------------------------------------------------- closed forms
-@pytest.mark.parametrize("variant", ["auto", "single", "split3"])
+@pytest.mark.parametrize("variant", ["auto", "single", "split3", "pair_k64"])
 @pytest.mark.parametrize("trans_b", [False, True])
 @pytest.mark.parametrize("M,N,K", [(300, 520, 2050), (256, 512, 8192), (70, 33, 9)])
 def test_ones_give_exactly_K(M, N, K, trans_b, variant):
@@ -187,7 +188,7 @@ def test_all_negative_product_is_zero(trans_b):
     assert (C.float() == 0).all()
 
 
-@pytest.mark.parametrize("variant", ["auto", "single", "split3", "packed"])
+@pytest.mark.parametrize("variant", ["auto", "single", "split3", "packed", "pair_k64"])
 @pytest.mark.parametrize("trans_b", [False, True])
 @pytest.mark.parametrize("in_dtype", [F16, BF16])
 @pytest.mark.parametrize("M,N,K", [(300, 520, 1000), (129, 264, 72), (5000 // 8, 3001, 2050)])

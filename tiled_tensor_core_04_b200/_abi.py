@@ -52,6 +52,7 @@ class GemmOptions(ctypes.Structure):
         ("force_pack", ctypes.c_int),
         ("max_ctas", ctypes.c_int),
         ("timeout_ns", ctypes.c_uint64),
+        ("stage_k", ctypes.c_int),
     ]
 
 

@@ -83,13 +83,23 @@ constexpr int kBN = 256;       // MMA N (tile columns)
 constexpr int kBK = 64;        // K per pipeline stage (128 bytes of 16-bit data)
 constexpr uint32_t kTmemCols = 512;
 
-template <bool PAIR>
+// PAIR: 2-CTA (cta_group::2) tile of 256 x 256, else 1-CTA tile of 128 x 256.
+// KK: 64-wide K sub-blocks per pipeline stage (stage K = 64 * KK).  Each
+// sub-block of A is one 128-row x 128-byte TMA box (16 KB, 128-byte swizzle);
+// B sub-blocks hold the CTA's kBNCta columns for the same 64 K.
+template <bool PAIR, int KK>
 struct TileCfg {
     static constexpr int kBNCta = PAIR ? kBN / 2 : kBN;           // B columns held per CTA
-    static constexpr int kABytes = kBM * kBK * 2;                  // 16 KB
-    static constexpr int kBBytes = kBNCta * kBK * 2;               // 16 or 32 KB
+    static constexpr int kStageK = kBK * KK;
+    static constexpr int kASub = kBM * kBK * 2;                    // 16 KB
+    static constexpr int kBSub = kBNCta * kBK * 2;                 // 16 or 32 KB
+    static constexpr int kABytes = KK * kASub;
+    static constexpr int kBBytes = KK * kBSub;
     static constexpr int kStageBytes = kABytes + kBBytes;
-    static constexpr int kStages = PAIR ? 7 : 4;
+    // as many stages as fit in 227 KB next to 1 KB of static shared memory
+    // and 1 KB of alignment slack (at most 8)
+    static constexpr int kStagesFit = (232448 - 2048) / kStageBytes;
+    static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
     static constexpr uint32_t kTxBytes = kStageBytes * (PAIR ? 2 : 1);
     static constexpr int kTileM = PAIR ? 2 * kBM : kBM;
     static constexpr int kSmemBytes = kStages * kStageBytes + 1024;  // + alignment slack
@@ -155,6 +165,31 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, const 
         }
     }
     return __all_sync(0xffffffffu, ok);
+}
+
+// Bounded wait executed by ONE thread (the TMA producer and MMA issuer run on
+// a single elected lane, so their waits carry no warp-wide vote).  Same
+// return convention as wait_phase.
+template <bool CLUSTER_SCOPE>
+__device__ __forceinline__ bool wait_phase_thread(uint32_t bar, uint32_t parity,
+                                                  const WaitCtx &wc, uint32_t code)
+{
+    auto probe = [&]() {
+        return CLUSTER_SCOPE ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
+    };
+    if (probe()) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t n = 1;; ++n) {
+        if (probe()) return true;
+        if ((n & 15u) == 0u) {
+            if (*reinterpret_cast<volatile int *>(wc.abort_flag)) return false;
+            if (global_timer_ns() - t0 > wc.timeout_ns) {
+                *reinterpret_cast<volatile int *>(wc.abort_flag) = 1;
+                atomicOr(&g_gemm_device_error, code);
+                return false;
+            }
+        }
+    }
 }
 
 // Single-thread bounded wait used only while tearing down after an abort.
@@ -226,12 +261,12 @@ __device__ __forceinline__ void store_row32(OutT *dst, const uint32_t (&v)[32], 
 }
 
 // ------------------------------------------------------------------ kernel
-template <bool PAIR, bool B_MN, typename OutT>
+template <bool PAIR, int KK, bool B_MN, typename OutT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_relu_tc_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB, const GemmParams p)
 {
-    using Cfg = TileCfg<PAIR>;
+    using Cfg = TileCfg<PAIR, KK>;
     constexpr int CG = PAIR ? 2 : 1;
     constexpr int kStages = Cfg::kStages;
 
@@ -284,119 +319,143 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool aborted = false;
 
     if (warp == 0) {
-        // ------------------------------------------------ TMA producer
-        int stage = 0;
-        uint32_t phase = 0;
-        uint32_t issued_mask = 0;  // stages that received at least one load
-        uint32_t last_parity = 0;  // parity of the last phase issued per stage (bit s)
-        for (int u = cluster_id; u < p.num_units && !aborted; u += num_clusters) {
-            const WorkUnit w = decode_unit(u, p.tiles_m, p.tiles_n, p.splits, p.kblocks, p.panel);
-            const int m_row = w.m_tile * Cfg::kTileM + static_cast<int>(rank) * kBM;
-            const int n_col = w.n_tile * kBN + static_cast<int>(rank) * Cfg::kBNCta;
-            for (int kb = w.kb0; kb < w.kb1; ++kb) {
-                if (!wait_phase<PAIR>(smem_addr(&empty_bar[stage]), phase ^ 1u, wc, kErrProducer)) {
-                    aborted = true;
-                    break;
-                }
-                if (lane == 0) {
+        // ------------------------------------------------ TMA producer (one lane)
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued_mask = 0;  // stages that received at least one load
+            uint32_t last_parity = 0;  // parity of the last phase issued per stage (bit s)
+            for (int u = cluster_id; u < p.num_units && !aborted; u += num_clusters) {
+                const WorkUnit w = decode_unit(u, p.tiles_m, p.tiles_n, p.splits, p.kblocks, p.panel);
+                const int m_row = w.m_tile * Cfg::kTileM + static_cast<int>(rank) * kBM;
+                const int n_col = w.n_tile * kBN + static_cast<int>(rank) * Cfg::kBNCta;
+                for (int kb = w.kb0; kb < w.kb1; ++kb) {
+                    // the slot is released by the MMA's tcgen05.commit (local in both CTAs)
+                    if (!wait_phase_thread<false>(smem_addr(&empty_bar[stage]), phase ^ 1u, wc,
+                                                  kErrProducer)) {
+                        aborted = true;
+                        break;
+                    }
                     const uint32_t fb = smem_addr(&full_bar[stage]);
                     const uint32_t a_dst = tiles_base + static_cast<uint32_t>(stage * Cfg::kStageBytes);
                     const uint32_t b_dst = a_dst + Cfg::kABytes;
-                    const int k0 = kb * kBK;
+                    const int k0 = kb * Cfg::kStageK;
                     if constexpr (PAIR) {
                         const uint32_t fb_leader = map_shared_to_rank(fb, 0);
                         if (rank == 0) mbar_arrive_expect_tx(fb, Cfg::kTxBytes);
-                        tma_load_2d_pair(a_dst, &tmA, fb_leader, k0, m_row);
-                        if constexpr (B_MN) {
 #pragma unroll
-                            for (int c = 0; c < Cfg::kBNCta / 64; ++c)
-                                tma_load_2d_pair(b_dst + c * 8192, &tmB, fb_leader, n_col + c * 64, k0);
-                        } else {
-                            tma_load_2d_pair(b_dst, &tmB, fb_leader, k0, n_col);
+                        for (int kk = 0; kk < KK; ++kk) {
+                            const int kx = k0 + kk * kBK;
+                            tma_load_2d_pair(a_dst + kk * Cfg::kASub, &tmA, fb_leader, kx, m_row);
+                            if constexpr (B_MN) {
+#pragma unroll
+                                for (int c = 0; c < Cfg::kBNCta / 64; ++c)
+                                    tma_load_2d_pair(b_dst + kk * Cfg::kBSub + c * 8192, &tmB, fb_leader,
+                                                     n_col + c * 64, kx);
+                            } else {
+                                tma_load_2d_pair(b_dst + kk * Cfg::kBSub, &tmB, fb_leader, kx, n_col);
+                            }
                         }
                     } else {
                         mbar_arrive_expect_tx(fb, Cfg::kTxBytes);
-                        tma_load_2d(a_dst, &tmA, fb, k0, m_row);
-                        if constexpr (B_MN) {
 #pragma unroll
-                            for (int c = 0; c < Cfg::kBNCta / 64; ++c)
-                                tma_load_2d(b_dst + c * 8192, &tmB, fb, n_col + c * 64, k0);
-                        } else {
-                            tma_load_2d(b_dst, &tmB, fb, k0, n_col);
+                        for (int kk = 0; kk < KK; ++kk) {
+                            const int kx = k0 + kk * kBK;
+                            tma_load_2d(a_dst + kk * Cfg::kASub, &tmA, fb, kx, m_row);
+                            if constexpr (B_MN) {
+#pragma unroll
+                                for (int c = 0; c < Cfg::kBNCta / 64; ++c)
+                                    tma_load_2d(b_dst + kk * Cfg::kBSub + c * 8192, &tmB, fb,
+                                                n_col + c * 64, kx);
+                            } else {
+                                tma_load_2d(b_dst + kk * Cfg::kBSub, &tmB, fb, kx, n_col);
+                            }
                         }
                     }
-                }
-                __syncwarp();
-                issued_mask |= 1u << stage;
-                last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
-                if (++stage == kStages) {
-                    stage = 0;
-                    phase ^= 1u;
+                    issued_mask |= 1u << stage;
+                    last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
                 }
             }
+            if (aborted && (!PAIR || rank == 0)) {
+                // let copies still in flight land before the CTA goes away
+                for (int s = 0; s < kStages; ++s)
+                    if (issued_mask & (1u << s))
+                        if (!wait_phase_one(smem_addr(&full_bar[s]), (last_parity >> s) & 1u, 20000000ull))
+                            atomicOr(&g_gemm_device_error, kErrDrain);
+            }
         }
-        if (aborted && lane == 0 && (!PAIR || rank == 0)) {
-            // let copies still in flight land before the CTA goes away
-            for (int s = 0; s < kStages; ++s)
-                if (issued_mask & (1u << s))
-                    if (!wait_phase_one(smem_addr(&full_bar[s]), (last_parity >> s) & 1u, 20000000ull))
-                        atomicOr(&g_gemm_device_error, kErrDrain);
-        }
+        __syncwarp();
     } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
-        if (rank == 0) {
+        // ------------------------------------------------ MMA issuer (one lane of the leader)
+        if (rank == 0 && lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
             int local = 0;
             bool issued_any = false;
+            // Descriptors of stage 0, k = 0; a stage / K step only moves the
+            // start address (bits 0-13, in 16-byte units).
+            const uint64_t a_desc0 = smem_desc_sw128(tiles_base, 16, 1024);
+            const uint64_t b_desc0 = B_MN ? smem_desc_sw128(tiles_base + Cfg::kABytes, 8192, 1024)
+                                          : smem_desc_sw128(tiles_base + Cfg::kABytes, 16, 1024);
+            constexpr uint64_t kAStep = 32 >> 4;                  // 16 K elements of a K-major row
+            constexpr uint64_t kBStep = B_MN ? (2048 >> 4) : (32 >> 4);  // 16 K rows / elements
+            constexpr uint64_t kStageStep = Cfg::kStageBytes >> 4;
+            constexpr uint64_t kASubStep = Cfg::kASub >> 4;
+            constexpr uint64_t kBSubStep = Cfg::kBSub >> 4;
+            // whether the next slot's operands were seen to have landed (peeked
+            // before the current slot's MMAs are issued, so the barrier check
+            // does not sit between two MMA groups)
+            bool next_ready = mbar_test_wait(smem_addr(&full_bar[0]), 0);
             for (int u = cluster_id; u < p.num_units && !aborted; u += num_clusters, ++local) {
                 const WorkUnit w = decode_unit(u, p.tiles_m, p.tiles_n, p.splits, p.kblocks, p.panel);
                 const int buf = local & 1;
                 const uint32_t tphase = static_cast<uint32_t>(local >> 1) & 1u;
-                if (!wait_phase<PAIR>(smem_addr(&tempty_bar[buf]), tphase ^ 1u, wc, kErrMmaAccum)) {
+                // the accumulator is released by the epilogue warps of both CTAs
+                if (!wait_phase_thread<PAIR>(smem_addr(&tempty_bar[buf]), tphase ^ 1u, wc,
+                                             kErrMmaAccum)) {
                     aborted = true;
                     break;
                 }
                 tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kBN);
                 for (int kb = w.kb0; kb < w.kb1; ++kb) {
-                    if (!wait_phase<PAIR>(smem_addr(&full_bar[stage]), phase, wc, kErrMmaOperands)) {
+                    if (!next_ready &&
+                        !wait_phase_thread<false>(smem_addr(&full_bar[stage]), phase, wc,
+                                                  kErrMmaOperands)) {
                         aborted = true;
                         break;
                     }
-                    tc_fence_after_sync();
-                    if (lane == 0) {
-                        const uint32_t a_base = tiles_base + static_cast<uint32_t>(stage * Cfg::kStageBytes);
-                        const uint32_t b_base = a_base + Cfg::kABytes;
+                    const int next_stage = stage + 1 == kStages ? 0 : stage + 1;
+                    const uint32_t next_phase = next_stage == 0 ? phase ^ 1u : phase;
+                    next_ready = mbar_test_wait(smem_addr(&full_bar[next_stage]), next_phase);
+                    const uint64_t so = static_cast<uint64_t>(stage) * kStageStep;
 #pragma unroll
-                        for (int k = 0; k < kBK / 16; ++k) {
-                            const uint64_t ad = smem_desc_sw128(a_base + k * 32, 16, 1024);
-                            const uint64_t bd = B_MN ? smem_desc_sw128(b_base + k * 2048, 8192, 1024)
-                                                     : smem_desc_sw128(b_base + k * 32, 16, 1024);
-                            umma_f16<CG>(d_tmem, ad, bd, p.idesc, (kb > w.kb0 || k > 0) ? 1u : 0u);
-                        }
-                        if constexpr (PAIR)
-                            umma_commit_pair(smem_addr(&empty_bar[stage]), 0x3);
-                        else
-                            umma_commit(smem_addr(&empty_bar[stage]));
+                    for (int k = 0; k < KK * (kBK / 16); ++k) {
+                        const uint64_t sub = static_cast<uint64_t>(k / (kBK / 16));
+                        const uint64_t kin = static_cast<uint64_t>(k % (kBK / 16));
+                        umma_f16<CG>(d_tmem, a_desc0 + so + sub * kASubStep + kin * kAStep,
+                                     b_desc0 + so + sub * kBSubStep + kin * kBStep, p.idesc,
+                                     (kb > w.kb0 || k > 0) ? 1u : 0u);
                     }
-                    __syncwarp();
+                    if constexpr (PAIR)
+                        umma_commit_pair(smem_addr(&empty_bar[stage]), 0x3);
+                    else
+                        umma_commit(smem_addr(&empty_bar[stage]));
                     issued_any = true;
-                    if (++stage == kStages) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
+                    stage = next_stage;
+                    phase = next_phase;
                 }
                 if (aborted) break;
-                if (lane == 0) {
-                    if constexpr (PAIR)
-                        umma_commit_pair(smem_addr(&tfull_bar[buf]), 0x3);
-                    else
-                        umma_commit(smem_addr(&tfull_bar[buf]));
-                }
-                __syncwarp();
+                if constexpr (PAIR)
+                    umma_commit_pair(smem_addr(&tfull_bar[buf]), 0x3);
+                else
+                    umma_commit(smem_addr(&tfull_bar[buf]));
             }
-            if (aborted && issued_any && lane == 0) {
+            if (aborted && issued_any) {
                 // wait for the MMAs already issued before TMEM is released
                 if constexpr (PAIR)
                     umma_commit_pair(smem_addr(&drain_bar), 0x1);
@@ -406,6 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     atomicOr(&g_gemm_device_error, kErrDrain);
             }
         }
+        __syncwarp();
     } else {
         // ------------------------------------------------ epilogue (warps 2..5)
         const int q = warp & 3;  // TMEM lane quarter this warp may access
@@ -414,7 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const WorkUnit w = decode_unit(u, p.tiles_m, p.tiles_n, p.splits, p.kblocks, p.panel);
             const int buf = local & 1;
             const uint32_t tphase = static_cast<uint32_t>(local >> 1) & 1u;
-            if (!wait_phase<PAIR>(smem_addr(&tfull_bar[buf]), tphase, wc, kErrEpilogue)) {
+            if (!wait_phase<false>(smem_addr(&tfull_bar[buf]), tphase, wc, kErrEpilogue)) {
                 aborted = true;
                 break;
             }

@@ -37,25 +37,43 @@ gemm_status_t cuda_fail(cudaError_t e, const char *what)
 // ------------------------------------------------------------------ kernels
 using GemmKernelFn = void (*)(const CUtensorMap, const CUtensorMap, const GemmParams);
 
-template <bool PAIR, bool BMN>
+// Instantiated variants: (pair, KK) in {(1-CTA, 1), (pair, 1), (pair, 2)},
+// B K-major or MN-major, fp16 / bf16 / fp32 output.
+template <bool PAIR, int KK, bool BMN>
 GemmKernelFn pick_out(gemm_dtype_t out)
 {
     switch (out) {
-    case GEMM_F16: return gemm_relu_tc_kernel<PAIR, BMN, __half>;
-    case GEMM_BF16: return gemm_relu_tc_kernel<PAIR, BMN, __nv_bfloat16>;
-    default: return gemm_relu_tc_kernel<PAIR, BMN, float>;
+    case GEMM_F16: return gemm_relu_tc_kernel<PAIR, KK, BMN, __half>;
+    case GEMM_BF16: return gemm_relu_tc_kernel<PAIR, KK, BMN, __nv_bfloat16>;
+    default: return gemm_relu_tc_kernel<PAIR, KK, BMN, float>;
     }
 }
 
-GemmKernelFn pick_kernel(bool pair, bool b_mn, gemm_dtype_t out)
+GemmKernelFn pick_kernel(bool pair, int kk, bool b_mn, gemm_dtype_t out)
 {
-    if (pair) return b_mn ? pick_out<true, true>(out) : pick_out<true, false>(out);
-    return b_mn ? pick_out<false, true>(out) : pick_out<false, false>(out);
+    if (pair && kk == 2) return b_mn ? pick_out<true, 2, true>(out) : pick_out<true, 2, false>(out);
+    if (pair) return b_mn ? pick_out<true, 1, true>(out) : pick_out<true, 1, false>(out);
+    return b_mn ? pick_out<false, 1, true>(out) : pick_out<false, 1, false>(out);
 }
 
-int variant_index(bool pair, bool b_mn, gemm_dtype_t out)
+int smem_bytes(bool pair, int kk)
 {
-    return (pair ? 6 : 0) + (b_mn ? 3 : 0) + static_cast<int>(out);
+    if (pair && kk == 2) return TileCfg<true, 2>::kSmemBytes;
+    if (pair) return TileCfg<true, 1>::kSmemBytes;
+    return TileCfg<false, 1>::kSmemBytes;
+}
+
+int stage_count(bool pair, int kk)
+{
+    if (pair && kk == 2) return TileCfg<true, 2>::kStages;
+    if (pair) return TileCfg<true, 1>::kStages;
+    return TileCfg<false, 1>::kStages;
+}
+
+int variant_index(bool pair, int kk, bool b_mn, gemm_dtype_t out)
+{
+    const int shape = pair ? (kk == 2 ? 2 : 1) : 0;
+    return shape * 6 + (b_mn ? 3 : 0) + static_cast<int>(out);
 }
 
 // ------------------------------------------------------------------ devices
@@ -64,18 +82,18 @@ struct DeviceInfo {
     bool ok = false;
     int sms = 0;
     int max_pair_clusters = 0;
-    bool attr_set[12] = {};
+    bool attr_set[18] = {};
 };
 
 std::mutex g_dev_mutex;
 DeviceInfo g_dev[kMaxDevices];
 
-gemm_status_t ensure_kernel_attr(DeviceInfo &d, bool pair, bool b_mn, gemm_dtype_t out)
+gemm_status_t ensure_kernel_attr(DeviceInfo &d, bool pair, int kk, bool b_mn, gemm_dtype_t out)
 {
-    const int v = variant_index(pair, b_mn, out);
+    const int v = variant_index(pair, kk, b_mn, out);
     if (d.attr_set[v]) return GEMM_OK;
-    const int smem = pair ? TileCfg<true>::kSmemBytes : TileCfg<false>::kSmemBytes;
-    cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void *>(pick_kernel(pair, b_mn, out)),
+    const int smem = smem_bytes(pair, kk);
+    cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void *>(pick_kernel(pair, kk, b_mn, out)),
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
     d.attr_set[v] = true;
@@ -102,12 +120,12 @@ gemm_status_t device_info(DeviceInfo **out)
         d.sms = sms;
         if (d.ok) {
             // how many 2-CTA clusters of the pair kernel fit at once
-            gemm_status_t st = ensure_kernel_attr(d, true, false, GEMM_F16);
+            gemm_status_t st = ensure_kernel_attr(d, true, 1, false, GEMM_F16);
             if (st != GEMM_OK) return st;
             cudaLaunchConfig_t cfg = {};
             cfg.gridDim = dim3(2 * sms, 1, 1);
             cfg.blockDim = dim3(kThreads, 1, 1);
-            cfg.dynamicSmemBytes = TileCfg<true>::kSmemBytes;
+            cfg.dynamicSmemBytes = smem_bytes(true, 1);
             cudaLaunchAttribute attr[1];
             attr[0].id = cudaLaunchAttributeClusterDimension;
             attr[0].val.clusterDim.x = 2;
@@ -117,7 +135,7 @@ gemm_status_t device_info(DeviceInfo **out)
             cfg.numAttrs = 1;
             int clusters = 0;
             e = cudaOccupancyMaxActiveClusters(
-                &clusters, reinterpret_cast<const void *>(pick_kernel(true, false, GEMM_F16)), &cfg);
+                &clusters, reinterpret_cast<const void *>(pick_kernel(true, 1, false, GEMM_F16)), &cfg);
             if (e != cudaSuccess || clusters <= 0) clusters = sms / 2;
             d.max_pair_clusters = std::min(clusters, sms / 2);
         }
@@ -153,16 +171,16 @@ gemm_status_t make_plan(int64_t M, int64_t N, int64_t K, gemm_dtype_t in, gemm_d
     if (in != GEMM_F16 && in != GEMM_BF16) return GEMM_ERR_UNSUPPORTED_DTYPE;
     if (out != GEMM_F16 && out != GEMM_BF16 && out != GEMM_F32) return GEMM_ERR_UNSUPPORTED_DTYPE;
     // the kernels index rows/columns with 32-bit ints; TMA dims must be < 2^32
-    if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX - kBK) return GEMM_ERR_INVALID_ARG;
+    if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX - 2 * kBK) return GEMM_ERR_INVALID_ARG;
     gemm_relu_options_t o = {};
     if (opts) o = *opts;
-    if (o.cta_pair < 0 || o.cta_pair > 2 || o.split_k < 0 || o.panel < 0 || o.max_ctas < 0)
+    if (o.cta_pair < 0 || o.cta_pair > 2 || o.split_k < 0 || o.panel < 0 || o.max_ctas < 0 ||
+        (o.stage_k != 0 && o.stage_k != 64 && o.stage_k != 128))
         return GEMM_ERR_INVALID_ARG;
 
     gemm_relu_plan_t p = {};
     p.tile_n = kBN;
-    p.tile_k = kBK;
-    p.kblocks = static_cast<int>(ceil_div(K, kBK));
+    p.kblocks = static_cast<int>(ceil_div(K, kBK));  // 64-wide; re-counted below for the pair
     const int64_t tiles_n = ceil_div(N, kBN);
     const int64_t tiles1 = ceil_div(M, kBM) * tiles_n;  // 1-CTA tiling
 
@@ -187,6 +205,10 @@ gemm_status_t make_plan(int64_t M, int64_t N, int64_t K, gemm_dtype_t in, gemm_d
 
     p.cta_pair = pair ? 1 : 0;
     p.tile_m = pair ? 2 * kBM : kBM;
+    // the pair kernel takes 128 of K per pipeline stage unless asked for 64
+    const int kk = (pair && o.stage_k != 64) ? 2 : 1;
+    p.tile_k = kBK * kk;
+    p.kblocks = static_cast<int>(ceil_div(K, p.tile_k));
     const int64_t tiles_m = ceil_div(M, p.tile_m);
     const int64_t units = tiles_m * tiles_n * split;
     if (units > INT32_MAX) return GEMM_ERR_INVALID_ARG;
@@ -196,7 +218,7 @@ gemm_status_t make_plan(int64_t M, int64_t N, int64_t K, gemm_dtype_t in, gemm_d
     p.panel = o.panel > 0 ? o.panel : kDefaultPanel;
     if (p.tiles_m > 0) p.panel = std::min(p.panel, p.tiles_m);
     p.units = static_cast<int>(units);
-    p.stages = pair ? TileCfg<true>::kStages : TileCfg<false>::kStages;
+    p.stages = stage_count(pair, kk);
 
     int64_t grid;
     if (pair) {
@@ -403,6 +425,7 @@ gemm_status_t run(const void *A, const void *B, void *C, int64_t M, int64_t N, i
     }
 
     const bool pair = plan.cta_pair != 0;
+    const int kk = plan.tile_k / kBK;
     const bool b_mn = !trans_b;
     const int bn_cta = pair ? kBN / 2 : kBN;
     CUtensorMap tmA, tmB;
@@ -436,14 +459,14 @@ gemm_status_t run(const void *A, const void *B, void *C, int64_t M, int64_t N, i
 
     {
         std::lock_guard<std::mutex> lock(g_dev_mutex);
-        st = ensure_kernel_attr(*dev, pair, b_mn, kout);
+        st = ensure_kernel_attr(*dev, pair, kk, b_mn, kout);
     }
     if (st != GEMM_OK) return st;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(plan.grid_ctas), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = pair ? TileCfg<true>::kSmemBytes : TileCfg<false>::kSmemBytes;
+    cfg.dynamicSmemBytes = smem_bytes(pair, kk);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -452,7 +475,7 @@ gemm_status_t run(const void *A, const void *B, void *C, int64_t M, int64_t N, i
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pair ? 1 : 0;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, pick_kernel(pair, b_mn, kout), tmA, tmB, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, pick_kernel(pair, kk, b_mn, kout), tmA, tmB, p);
     if (e != cudaSuccess) return cuda_fail(e, "gemm kernel launch");
 
     if (split) {
@@ -691,17 +714,17 @@ extern "C" gemm_status_t gemm_relu_splitk_noalloc(const void *A, const void *B, 
     p.timeout_ns = kDefaultTimeoutNs;
     {
         std::lock_guard<std::mutex> lock(g_dev_mutex);
-        st = ensure_kernel_attr(*dev, false, b_mn, kout);
+        st = ensure_kernel_attr(*dev, false, 1, b_mn, kout);
     }
     if (st != GEMM_OK) return st;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(plan.grid_ctas), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = TileCfg<false>::kSmemBytes;
+    cfg.dynamicSmemBytes = smem_bytes(false, 1);
     cfg.stream = stream;
     cfg.numAttrs = 0;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, pick_kernel(false, b_mn, kout), tmA, tmB, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, pick_kernel(false, 1, b_mn, kout), tmA, tmB, p);
     if (e != cudaSuccess) return cuda_fail(e, "no-alloc gemm kernel launch");
     if (split) {
         const int64_t n_total = M * N;
