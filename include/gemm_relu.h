@@ -84,6 +84,14 @@ typedef struct {
     uint64_t timeout_ns; /* 0 = 1 s; bound on every in-kernel barrier wait                */
     int stage_k;         /* 0 = auto (128 for the CTA pair, 64 otherwise); 64 or 128: K per
                             shared-memory pipeline stage of the CTA-pair kernel            */
+    int l2_hint_a;       /* L2 eviction priority of A's tile loads: 0 normal, 1 evict-first,
+                            2 evict-last (the analogue of the Ascend kernel's l2_cache_ctrl) */
+    int l2_hint_b;       /* same for B                                                      */
+    int c_streaming;     /* 1 = write C with evict-first (streaming) stores                 */
+    uint32_t wait_sleep_ns; /* suspend-time hint (ns) of the epilogue's barrier waits; 0 =
+                            the hardware default                                        */
+    int swap_ab;         /* skinny-M kernel computing C^T = op(B)^T A^T: 0 = auto (M <= 64
+                            and cta_pair auto), 1 = use it (needs M <= 128), 2 = never     */
 } gemm_relu_options_t;
 /* cta_pair: 0 = auto, 1 = force the 2-CTA (256 x 256 tile, cta_group::2)
  * kernel, 2 = force the 1-CTA (128 x 256 tile) kernel.  Split-K always uses
@@ -104,6 +112,7 @@ typedef struct {
     int grid_ctas;       /* persistent grid size in CTAs                                  */
     int stages;          /* shared-memory pipeline depth                                  */
     int pack_a, pack_b;  /* 1 = operand is re-pitched into the workspace first            */
+    int swap_ab;         /* 1 = skinny-M kernel: tiles of tile_n columns of C, all M rows  */
     int64_t workspace_bytes;
 } gemm_relu_plan_t;
 

@@ -74,11 +74,16 @@ def test_plans_for_the_workloads(lib):
     assert p["kblocks"] == 17 and p["tiles_m"] == 20 and p["tiles_n"] == 12   # K tail 2050 % 128
 
     p = plan(wl.WORKLOADS["skinny64x8192x8192_f16"])
-    assert p["cta_pair"] == 0 and p["split_k"] == 4 and p["units"] == 128
-    assert p["workspace_bytes"] >= 4 * 64 * 8192 * 4
+    assert p["swap_ab"] == 1 and p["tile_m"] == 64 and p["tile_n"] == 128
+    assert p["tiles_n"] == 64 and p["split_k"] == 2 and p["units"] == 128
+    assert p["workspace_bytes"] >= 2 * 64 * 8192 * 4
 
     p = plan(wl.WORKLOADS["skinny16x16384x4096_f16"])
-    assert p["cta_pair"] == 0 and p["split_k"] == 2 and p["units"] == 128
+    assert p["swap_ab"] == 1 and p["tile_m"] == 16 and p["split_k"] == 1 and p["units"] == 128
+    assert p["workspace_bytes"] == 0
+    # the main kernel's split-K path for the same shape when swap-AB is off
+    p = plan(wl.WORKLOADS["skinny64x8192x8192_f16"], swap_ab=2)
+    assert p["swap_ab"] == 0 and p["cta_pair"] == 0 and p["split_k"] == 4
 
     p = plan(wl.WORKLOADS["square256_f16"])
     assert p["units"] == 1 and p["grid_ctas"] == 2
@@ -102,6 +107,18 @@ def test_options_override_the_plan(lib):
         plan(w, stage_k=96)
 
 
+@pytest.mark.parametrize("M,np_", [(1, 16), (16, 16), (17, 32), (32, 32), (33, 64), (64, 64),
+                                    (65, 128), (128, 128)])
+def test_swap_ab_bucket(lib, M, np_):
+    p = g.gemm_relu_plan(M, 4096, 4096, torch.float16, torch.float16, False,
+                         options={"swap_ab": 1})
+    assert p["swap_ab"] == 1 and p["tile_m"] == np_ and p["tiles_m"] == 1
+    auto = g.gemm_relu_plan(M, 4096, 4096, torch.float16, torch.float16, False)
+    assert auto["swap_ab"] == (1 if M <= 64 else 0)
+    assert g.gemm_relu_plan(129, 4096, 4096, torch.float16, torch.float16, False,
+                            options={"swap_ab": 1})["swap_ab"] == 0
+
+
 def test_misaligned_base_pointer_is_repitched(lib):
     p = g.gemm_relu_plan(512, 512, 512, torch.float16, torch.float16, False, A=0x1002, B=0x2000)
     assert p["pack_a"] == 1 and p["pack_b"] == 0
@@ -117,6 +134,8 @@ def test_misaligned_base_pointer_is_repitched(lib):
     (1000, 300, 130, {"cta_pair": g.GEMM_CTA_SINGLE, "panel": 5}),
     (257, 257, 65, {"panel": 1}),
     (600, 300, 1000, {"stage_k": 64}),
+    (64, 8192, 8192, {"swap_ab": 1}),
+    (100, 1000, 3000, {"swap_ab": 1, "split_k": 5}),
 ])
 def test_units_cover_every_tile_and_k_block_once(lib, M, N, K, opt):
     p = g.gemm_relu_plan(M, N, K, torch.float16, torch.float16, False, options=opt or None)

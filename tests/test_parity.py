@@ -98,6 +98,10 @@ VARIANTS = {
     "split3": {"split_k": 3},
     "packed": {"force_pack": 1},
     "few_ctas": {"max_ctas": 3, "panel": 2},
+    "l2_hints": {"l2_hint_a": 2, "l2_hint_b": 1, "c_streaming": 1, "wait_sleep_ns": 20000},
+    "swap": {"swap_ab": 1},
+    "swap_split3": {"swap_ab": 1, "split_k": 3},
+    "no_swap": {"swap_ab": 2},
 }
 
 
@@ -115,6 +119,23 @@ def test_shapes_fp16(M, N, K, trans_b, variant):
 @pytest.mark.parametrize("variant", ["auto", "single", "split3", "pair_k64"])
 def test_dtypes_and_relu(in_dtype, out_dtype, trans_b, relu, variant):
     full_case(300, 520, 330, in_dtype, out_dtype, trans_b, relu, VARIANTS[variant], seed=7,
+              dist="normal")
+
+
+@pytest.mark.parametrize("variant", ["swap", "swap_split3", "auto", "no_swap"])
+@pytest.mark.parametrize("trans_b", [False, True])
+@pytest.mark.parametrize("M", [1, 7, 16, 17, 33, 64, 65, 100, 128])
+def test_skinny_M(M, trans_b, variant):
+    full_case(M, 1000, 1100, F16, F16, trans_b, options=VARIANTS[variant], seed=M)
+
+
+@pytest.mark.parametrize("out_dtype", [F16, BF16, F32])
+@pytest.mark.parametrize("in_dtype", [F16, BF16])
+@pytest.mark.parametrize("relu", [True, False])
+def test_skinny_dtypes(in_dtype, out_dtype, relu):
+    full_case(40, 777, 520, in_dtype, out_dtype, True, relu, VARIANTS["swap"], seed=3,
+              dist="normal")
+    full_case(40, 776, 520, in_dtype, out_dtype, False, relu, VARIANTS["swap_split3"], seed=4,
               dist="normal")
 
 

@@ -53,13 +53,18 @@ class GemmOptions(ctypes.Structure):
         ("max_ctas", ctypes.c_int),
         ("timeout_ns", ctypes.c_uint64),
         ("stage_k", ctypes.c_int),
+        ("l2_hint_a", ctypes.c_int),
+        ("l2_hint_b", ctypes.c_int),
+        ("c_streaming", ctypes.c_int),
+        ("wait_sleep_ns", ctypes.c_uint32),
+        ("swap_ab", ctypes.c_int),
     ]
 
 
 class GemmPlan(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "cta_pair", "tile_m", "tile_n", "tile_k", "tiles_m", "tiles_n", "kblocks", "split_k",
-        "panel", "units", "grid_ctas", "stages", "pack_a", "pack_b")] + [
+        "panel", "units", "grid_ctas", "stages", "pack_a", "pack_b", "swap_ab")] + [
         ("workspace_bytes", ctypes.c_int64)]
 
     def as_dict(self) -> dict:

@@ -81,7 +81,7 @@ __global__ void selftest_timeout_kernel(uint64_t timeout_ns, int *out)
         fence_barrier_init();
     }
     __syncthreads();
-    const WaitCtx wc{&abort_flag, timeout_ns};
+    const WaitCtx wc{&abort_flag, timeout_ns, 1000};
     const bool ok = wait_phase<false>(smem_addr(&bar), 0, wc, kErrSelfTest);
     if (threadIdx.x == 0) out[0] = ok ? 1 : 0;
 }

@@ -75,6 +75,9 @@ struct GemmParams {
     int vec_ok;            // 16-byte vector stores are aligned
     uint32_t idesc;        // tcgen05 instruction descriptor
     uint64_t timeout_ns;
+    int l2_a, l2_b;        // L2 eviction priority of the A / B loads (0 normal, 1 first, 2 last)
+    int c_stream;          // 1: store C with evict-first (streaming) stores
+    uint32_t sleep_ns;     // suspend-time hint for the epilogue's accumulator waits
 };
 
 constexpr int kThreads = 192;  // 6 warps
@@ -133,6 +136,7 @@ __host__ __device__ __forceinline__ WorkUnit decode_unit(int u, int tiles_m, int
 struct WaitCtx {
     int *abort_flag;  // shared, per CTA
     uint64_t timeout_ns;
+    uint32_t sleep_ns;  // suspend-time hint of the warp-wide (epilogue) waits
 };
 
 // Bounded wait on an mbarrier phase, executed by all 32 lanes of a warp.
@@ -144,7 +148,9 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, const 
                                            uint32_t code)
 {
     auto probe = [&]() {
-        return CLUSTER_SCOPE ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
+        if (CLUSTER_SCOPE) return mbar_try_wait_cluster(bar, parity);
+        return wc.sleep_ns ? mbar_try_wait_sleep(bar, parity, wc.sleep_ns)
+                           : mbar_try_wait(bar, parity);
     };
     bool ok = probe();
     if (!ok) {
@@ -230,7 +236,7 @@ __device__ __forceinline__ OutT convert_out(float x)
 // range.  `vec`: the destination is 16-byte aligned.
 template <typename OutT>
 __device__ __forceinline__ void store_row32(OutT *dst, const uint32_t (&v)[32], int valid,
-                                            bool vec, int relu)
+                                            bool vec, int relu, bool stream)
 {
     float f[32];
 #pragma unroll
@@ -242,16 +248,26 @@ __device__ __forceinline__ void store_row32(OutT *dst, const uint32_t (&v)[32], 
         if constexpr (std::is_same_v<OutT, float>) {
             float4 *d4 = reinterpret_cast<float4 *>(dst);
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                d4[i] = make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
+            for (int i = 0; i < 8; ++i) {
+                const float4 q = make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]);
+                if (stream)
+                    __stcs(d4 + i, q);
+                else
+                    d4[i] = q;
+            }
         } else {
             uint4 *d4 = reinterpret_cast<uint4 *>(dst);
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-                d4[i] = make_uint4(pack_pair<OutT>(f[8 * i + 0], f[8 * i + 1]),
-                                   pack_pair<OutT>(f[8 * i + 2], f[8 * i + 3]),
-                                   pack_pair<OutT>(f[8 * i + 4], f[8 * i + 5]),
-                                   pack_pair<OutT>(f[8 * i + 6], f[8 * i + 7]));
+            for (int i = 0; i < 4; ++i) {
+                const uint4 q = make_uint4(pack_pair<OutT>(f[8 * i + 0], f[8 * i + 1]),
+                                           pack_pair<OutT>(f[8 * i + 2], f[8 * i + 3]),
+                                           pack_pair<OutT>(f[8 * i + 4], f[8 * i + 5]),
+                                           pack_pair<OutT>(f[8 * i + 6], f[8 * i + 7]));
+                if (stream)
+                    __stcs(d4 + i, q);
+                else
+                    d4[i] = q;
+            }
         }
     } else {
 #pragma unroll
@@ -313,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after_sync();
     const uint32_t tmem_base = tmem_slot;
 
-    const WaitCtx wc{&abort_flag, p.timeout_ns};
+    const WaitCtx wc{&abort_flag, p.timeout_ns, p.sleep_ns};
     const int cluster_id = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
     const int num_clusters = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
     bool aborted = false;
@@ -321,6 +337,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         // ------------------------------------------------ TMA producer (one lane)
         if (lane == 0) {
+            const uint64_t pol_a = make_l2_policy(p.l2_a);
+            const uint64_t pol_b = make_l2_policy(p.l2_b);
             int stage = 0;
             uint32_t phase = 0;
             uint32_t issued_mask = 0;  // stages that received at least one load
@@ -346,14 +364,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int kk = 0; kk < KK; ++kk) {
                             const int kx = k0 + kk * kBK;
-                            tma_load_2d_pair(a_dst + kk * Cfg::kASub, &tmA, fb_leader, kx, m_row);
+                            tma_load_2d_pair_hint(a_dst + kk * Cfg::kASub, &tmA, fb_leader, kx, m_row,
+                                                  pol_a);
                             if constexpr (B_MN) {
 #pragma unroll
                                 for (int c = 0; c < Cfg::kBNCta / 64; ++c)
-                                    tma_load_2d_pair(b_dst + kk * Cfg::kBSub + c * 8192, &tmB, fb_leader,
-                                                     n_col + c * 64, kx);
+                                    tma_load_2d_pair_hint(b_dst + kk * Cfg::kBSub + c * 8192, &tmB,
+                                                          fb_leader, n_col + c * 64, kx, pol_b);
                             } else {
-                                tma_load_2d_pair(b_dst + kk * Cfg::kBSub, &tmB, fb_leader, kx, n_col);
+                                tma_load_2d_pair_hint(b_dst + kk * Cfg::kBSub, &tmB, fb_leader, kx,
+                                                      n_col, pol_b);
                             }
                         }
                     } else {
@@ -361,14 +381,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int kk = 0; kk < KK; ++kk) {
                             const int kx = k0 + kk * kBK;
-                            tma_load_2d(a_dst + kk * Cfg::kASub, &tmA, fb, kx, m_row);
+                            tma_load_2d_hint(a_dst + kk * Cfg::kASub, &tmA, fb, kx, m_row, pol_a);
                             if constexpr (B_MN) {
 #pragma unroll
                                 for (int c = 0; c < Cfg::kBNCta / 64; ++c)
-                                    tma_load_2d(b_dst + kk * Cfg::kBSub + c * 8192, &tmB, fb,
-                                                n_col + c * 64, kx);
+                                    tma_load_2d_hint(b_dst + kk * Cfg::kBSub + c * 8192, &tmB, fb,
+                                                     n_col + c * 64, kx, pol_b);
                             } else {
-                                tma_load_2d(b_dst + kk * Cfg::kBSub, &tmB, fb, kx, n_col);
+                                tma_load_2d_hint(b_dst + kk * Cfg::kBSub, &tmB, fb, kx, n_col, pol_b);
                             }
                         }
                     }
@@ -493,7 +513,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_load_32cols(taddr + static_cast<uint32_t>(c), v);
                 tmem_load_wait();
                 const int valid = min(32, p.N - (col0 + c));
-                if (row_ok) store_row32<OutT>(rowp + c, v, valid, p.vec_ok != 0, p.relu);
+                if (row_ok) store_row32<OutT>(rowp + c, v, valid, p.vec_ok != 0, p.relu, p.c_stream != 0);
             }
             tc_fence_before_sync();
             __syncwarp();

@@ -16,6 +16,7 @@
 #include "../../include/gemm_relu.h"
 #include "aux_kernels.cuh"
 #include "gemm_kernel.cuh"
+#include "skinny_kernel.cuh"
 
 namespace {
 
@@ -76,6 +77,60 @@ int variant_index(bool pair, int kk, bool b_mn, gemm_dtype_t out)
     return shape * 6 + (b_mn ? 3 : 0) + static_cast<int>(out);
 }
 
+// Skinny-M (swap-AB) kernels: NP in {16, 32, 64, 128}, B MN- or K-major.
+template <int NP, bool BMN>
+GemmKernelFn pick_skinny_out(gemm_dtype_t out)
+{
+    switch (out) {
+    case GEMM_F16: return gemm_relu_skinny_kernel<NP, BMN, __half>;
+    case GEMM_BF16: return gemm_relu_skinny_kernel<NP, BMN, __nv_bfloat16>;
+    default: return gemm_relu_skinny_kernel<NP, BMN, float>;
+    }
+}
+
+template <bool BMN>
+GemmKernelFn pick_skinny_np(int np, gemm_dtype_t out)
+{
+    switch (np) {
+    case 16: return pick_skinny_out<16, BMN>(out);
+    case 32: return pick_skinny_out<32, BMN>(out);
+    case 64: return pick_skinny_out<64, BMN>(out);
+    default: return pick_skinny_out<128, BMN>(out);
+    }
+}
+
+GemmKernelFn pick_skinny(int np, bool b_mn, gemm_dtype_t out)
+{
+    return b_mn ? pick_skinny_np<true>(np, out) : pick_skinny_np<false>(np, out);
+}
+
+int skinny_smem(int np)
+{
+    switch (np) {
+    case 16: return SkinnyCfg<16>::kSmemBytes;
+    case 32: return SkinnyCfg<32>::kSmemBytes;
+    case 64: return SkinnyCfg<64>::kSmemBytes;
+    default: return SkinnyCfg<128>::kSmemBytes;
+    }
+}
+
+int skinny_stages(int np)
+{
+    switch (np) {
+    case 16: return SkinnyCfg<16>::kStages;
+    case 32: return SkinnyCfg<32>::kStages;
+    case 64: return SkinnyCfg<64>::kStages;
+    default: return SkinnyCfg<128>::kStages;
+    }
+}
+
+// index of a skinny variant in DeviceInfo::skinny_attr_set
+int skinny_index(int np, bool b_mn, gemm_dtype_t out)
+{
+    const int npi = np == 16 ? 0 : np == 32 ? 1 : np == 64 ? 2 : 3;
+    return npi * 6 + (b_mn ? 3 : 0) + static_cast<int>(out);
+}
+
 // ------------------------------------------------------------------ devices
 struct DeviceInfo {
     bool ready = false;
@@ -83,6 +138,7 @@ struct DeviceInfo {
     int sms = 0;
     int max_pair_clusters = 0;
     bool attr_set[18] = {};
+    bool skinny_attr_set[24] = {};
 };
 
 std::mutex g_dev_mutex;
@@ -97,6 +153,18 @@ gemm_status_t ensure_kernel_attr(DeviceInfo &d, bool pair, int kk, bool b_mn, ge
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
     d.attr_set[v] = true;
+    return GEMM_OK;
+}
+
+gemm_status_t ensure_skinny_attr(DeviceInfo &d, int np, bool b_mn, gemm_dtype_t out)
+{
+    const int v = skinny_index(np, b_mn, out);
+    if (d.skinny_attr_set[v]) return GEMM_OK;
+    cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void *>(pick_skinny(np, b_mn, out)),
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         skinny_smem(np));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(skinny)");
+    d.skinny_attr_set[v] = true;
     return GEMM_OK;
 }
 
@@ -175,7 +243,8 @@ gemm_status_t make_plan(int64_t M, int64_t N, int64_t K, gemm_dtype_t in, gemm_d
     gemm_relu_options_t o = {};
     if (opts) o = *opts;
     if (o.cta_pair < 0 || o.cta_pair > 2 || o.split_k < 0 || o.panel < 0 || o.max_ctas < 0 ||
-        (o.stage_k != 0 && o.stage_k != 64 && o.stage_k != 128))
+        (o.stage_k != 0 && o.stage_k != 64 && o.stage_k != 128) || o.l2_hint_a < 0 ||
+        o.l2_hint_a > 2 || o.l2_hint_b < 0 || o.l2_hint_b > 2 || o.c_streaming < 0 || o.c_streaming > 1 || o.swap_ab < 0 || o.swap_ab > 2)
         return GEMM_ERR_INVALID_ARG;
 
     gemm_relu_plan_t p = {};
@@ -183,6 +252,39 @@ gemm_status_t make_plan(int64_t M, int64_t N, int64_t K, gemm_dtype_t in, gemm_d
     p.kblocks = static_cast<int>(ceil_div(K, kBK));  // 64-wide; re-counted below for the pair
     const int64_t tiles_n = ceil_div(N, kBN);
     const int64_t tiles1 = ceil_div(M, kBM) * tiles_n;  // 1-CTA tiling
+
+    // skinny M: the transposed product on the swap-AB kernel (M <= 128 only)
+    const bool swap = M <= 128 && M > 0 &&
+                      (o.swap_ab == 1 || (o.swap_ab == 0 && M <= 64 && o.cta_pair == GEMM_CTA_AUTO));
+    if (swap) {
+        const int np = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+        p.swap_ab = 1;
+        p.cta_pair = 0;
+        p.tile_m = np;
+        p.tile_n = 128;
+        p.tile_k = kBK;
+        p.tiles_m = 1;
+        p.tiles_n = static_cast<int>(ceil_div(N, 128));
+        int64_t sp = o.split_k;
+        if (sp == 0) {
+            sp = 1;
+            if (p.tiles_n * 2 <= num_sms && p.kblocks >= 8) {
+                sp = std::max<int64_t>(1, num_sms / p.tiles_n);
+                sp = std::min<int64_t>(sp, p.kblocks / 4);
+                sp = std::min<int64_t>(sp, 32);
+            }
+        }
+        sp = p.kblocks > 0 ? std::max<int64_t>(1, std::min<int64_t>(sp, p.kblocks)) : 1;
+        const int64_t su = static_cast<int64_t>(p.tiles_n) * sp;
+        if (su > INT32_MAX) return GEMM_ERR_INVALID_ARG;
+        p.split_k = static_cast<int>(sp);
+        p.panel = 1;
+        p.units = static_cast<int>(su);
+        p.stages = skinny_stages(np);
+        int64_t ctas = num_sms;
+        if (o.max_ctas > 0) ctas = std::min<int64_t>(ctas, o.max_ctas);
+        p.grid_ctas = static_cast<int>(std::min<int64_t>(su, ctas));
+    }
 
     int64_t split = o.split_k;
     if (split == 0) {
@@ -197,6 +299,7 @@ gemm_status_t make_plan(int64_t M, int64_t N, int64_t K, gemm_dtype_t in, gemm_d
     if (p.kblocks > 0) split = std::max<int64_t>(1, std::min<int64_t>(split, p.kblocks));
     else split = 1;
 
+    if (!swap) {
     bool pair;
     if (split > 1) pair = false;
     else if (o.cta_pair == GEMM_CTA_PAIR) pair = true;
@@ -231,6 +334,7 @@ gemm_status_t make_plan(int64_t M, int64_t N, int64_t K, gemm_dtype_t in, gemm_d
         grid = std::min<int64_t>(units, ctas);
     }
     p.grid_ctas = static_cast<int>(grid);
+    }  // !swap
 
     // TMA reads rows whose byte pitch and base address are 16-byte aligned
     const int64_t a_row_bytes = K * 2;
@@ -349,10 +453,10 @@ gemm_status_t encode_2d(CUtensorMap *map, const void *base, gemm_dtype_t dt, int
 // tcgen05 instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A/B type
 // (bits 7-9 / 10-12: 0 fp16, 1 bf16), A K-major (bit 15 = 0), B major (bit
 // 16: 0 K-major, 1 MN-major), N >> 3 (bits 17-22), M >> 4 (bits 24-28).
-uint32_t make_idesc(gemm_dtype_t in, bool b_mn, int mma_m, int mma_n)
+uint32_t make_idesc(gemm_dtype_t in, bool b_mn, int mma_m, int mma_n, bool a_mn = false)
 {
     const uint32_t t = in == GEMM_BF16 ? 1u : 0u;
-    return (1u << 4) | (t << 7) | (t << 10) | ((b_mn ? 1u : 0u) << 16) |
+    return (1u << 4) | (t << 7) | (t << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
            (static_cast<uint32_t>(mma_n >> 3) << 17) | (static_cast<uint32_t>(mma_m >> 4) << 24);
 }
 
@@ -374,6 +478,77 @@ void launch_reduce_t(const float *ws, void *C, int64_t n_total, int splits, int6
 {
     splitk_reduce_kernel<OutT><<<grid, 256, 0, stream>>>(ws, static_cast<OutT *>(C), n_total,
                                                           splits, split_stride, relu, vec4);
+}
+
+// Skinny-M path: C^T tiles on the swap-AB kernel (+ the split-K reduction).
+gemm_status_t launch_skinny(const gemm_relu_plan_t &plan, const void *a_src, int64_t a_pitch,
+                            const void *b_src, int64_t b_pitch, void *C, int64_t M, int64_t N,
+                            int64_t K, gemm_dtype_t in, gemm_dtype_t out, int trans_b, int relu,
+                            void *split_ws, const gemm_relu_options_t *opts, DeviceInfo *dev,
+                            cudaStream_t stream)
+{
+    const int np = plan.tile_m;
+    const bool b_mn = !trans_b;
+    CUtensorMap tmA, tmB;
+    gemm_status_t st = encode_2d(&tmA, a_src, in, K, M, a_pitch, kBK, np);
+    if (st != GEMM_OK) return st;
+    if (b_mn)
+        st = encode_2d(&tmB, b_src, in, N, K, b_pitch, 64, kBK);
+    else
+        st = encode_2d(&tmB, b_src, in, K, N, b_pitch, kBK, 128);
+    if (st != GEMM_OK) return st;
+
+    const bool split = plan.split_k > 1;
+    const gemm_dtype_t kout = split ? GEMM_F32 : out;
+    GemmParams p = {};
+    p.C = split ? split_ws : C;
+    p.ldc = N;
+    p.split_stride = split ? M * N : 0;
+    p.M = static_cast<int>(M);
+    p.N = static_cast<int>(N);
+    p.K = static_cast<int>(K);
+    p.tiles_m = plan.tiles_m;
+    p.tiles_n = plan.tiles_n;
+    p.splits = plan.split_k;
+    p.kblocks = plan.kblocks;
+    p.panel = plan.panel;
+    p.num_units = plan.units;
+    p.relu = split ? 0 : (relu ? 1 : 0);
+    p.vec_ok = 0;
+    // MMA: 128 columns of C (op(B)^T, MN-major when B is stored (K, N)) x np rows of C
+    p.idesc = make_idesc(in, false, 128, np, b_mn);
+    p.timeout_ns = (opts && opts->timeout_ns) ? opts->timeout_ns : kDefaultTimeoutNs;
+    p.l2_a = opts ? opts->l2_hint_a : 0;
+    p.l2_b = opts ? opts->l2_hint_b : 0;
+    p.sleep_ns = (opts && opts->wait_sleep_ns) ? opts->wait_sleep_ns : 0;
+    {
+        std::lock_guard<std::mutex> lock(g_dev_mutex);
+        st = ensure_skinny_attr(*dev, np, b_mn, kout);
+    }
+    if (st != GEMM_OK) return st;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(plan.grid_ctas), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = skinny_smem(np);
+    cfg.stream = stream;
+    cfg.numAttrs = 0;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, pick_skinny(np, b_mn, kout), tmA, tmB, p);
+    if (e != cudaSuccess) return cuda_fail(e, "skinny gemm kernel launch");
+    if (split) {
+        const int64_t n_total = M * N;
+        const int vec4 = (n_total % 4) == 0 ? 1 : 0;
+        const int grid = static_cast<int>(std::min<int64_t>(ceil_div(n_total / (vec4 ? 4 : 1), 256),
+                                                            static_cast<int64_t>(dev->sms) * 8));
+        const float *wsf = static_cast<const float *>(split_ws);
+        switch (out) {
+        case GEMM_F16: launch_reduce_t<__half>(wsf, C, n_total, plan.split_k, M * N, relu ? 1 : 0, vec4, grid, stream); break;
+        case GEMM_BF16: launch_reduce_t<__nv_bfloat16>(wsf, C, n_total, plan.split_k, M * N, relu ? 1 : 0, vec4, grid, stream); break;
+        default: launch_reduce_t<float>(wsf, C, n_total, plan.split_k, M * N, relu ? 1 : 0, vec4, grid, stream); break;
+        }
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "split-K reduce launch");
+    }
+    return GEMM_OK;
 }
 
 gemm_status_t run(const void *A, const void *B, void *C, int64_t M, int64_t N, int64_t K,
@@ -424,6 +599,10 @@ gemm_status_t run(const void *A, const void *B, void *C, int64_t M, int64_t N, i
         b_pitch = lay.b_pitch;
     }
 
+    if (plan.swap_ab)
+        return launch_skinny(plan, a_src, a_pitch, b_src, b_pitch, C, M, N, K, in, out, trans_b,
+                             relu, wsb + lay.split_off, opts, dev, stream);
+
     const bool pair = plan.cta_pair != 0;
     const int kk = plan.tile_k / kBK;
     const bool b_mn = !trans_b;
@@ -456,6 +635,10 @@ gemm_status_t run(const void *A, const void *B, void *C, int64_t M, int64_t N, i
     p.vec_ok = (!misaligned16(p.C) && ((N * static_cast<int64_t>(dtype_size(kout))) % 16) == 0) ? 1 : 0;
     p.idesc = make_idesc(in, b_mn, pair ? 2 * kBM : kBM, kBN);
     p.timeout_ns = (opts && opts->timeout_ns) ? opts->timeout_ns : kDefaultTimeoutNs;
+    p.l2_a = opts ? opts->l2_hint_a : 0;
+    p.l2_b = opts ? opts->l2_hint_b : 0;
+    p.c_stream = (!split && opts) ? opts->c_streaming : 0;
+    p.sleep_ns = (opts && opts->wait_sleep_ns) ? opts->wait_sleep_ns : 0;
 
     {
         std::lock_guard<std::mutex> lock(g_dev_mutex);
@@ -655,6 +838,7 @@ extern "C" gemm_status_t gemm_relu_splitk_noalloc(const void *A, const void *B, 
     gemm_relu_options_t o = {};
     o.cta_pair = GEMM_CTA_SINGLE;
     o.split_k = split_k;
+    o.swap_ab = 2;
     gemm_relu_plan_t plan;
     Layout lay;
     gemm_status_t st = make_plan(M, N, K, in, out, trans_b, A, B, 148, 74, &o, &plan, &lay);

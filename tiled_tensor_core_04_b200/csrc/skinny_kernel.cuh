@@ -1,0 +1,253 @@
+// skinny_kernel.cuh -- fused GEMM + ReLU for skinny M (M <= 128), computed as
+// the transposed product:  C^T = op(B)^T . A^T.
+//
+// For a short M the 128-row MMA of the main kernel would mostly multiply the
+// zero rows TMA fills in, and its 48 KB pipeline stages leave only four
+// stages of loads in flight, while the problem is bound by streaming B from
+// HBM.  Here the MMA's 128-row side runs over N (128 columns of C per tile)
+// and its N side over all of M (NP = 16, 32, 64 or 128 >= M), so every MMA
+// row is useful and a stage holds only the B tile (16 KB) plus NP x 64 of A,
+// which keeps 8-12 stages of B in flight per SM.
+//
+//   MMA "A" operand (128 x 64 per stage): op(B)^T tile.  B stored (K, N) is
+//     N-contiguous -> MN-major operand (two 64-column TMA boxes); B stored
+//     (N, K) is K-contiguous -> K-major operand (one 64 x 128 box).
+//   MMA "B" operand (NP x 64): the A rows, K-major (one 64 x NP box; rows
+//     past M read as zero).
+//   Accumulator: TMEM lane = column n of C, TMEM column = row m of C; two
+//     NP-column buffers so the epilogue overlaps the next tile.
+//   Epilogue: lane t of warp q holds C[:, n0 + 32q + t]; for each m it writes
+//     C[m, n] -- 32 consecutive n per warp store, i.e. coalesced rows of C.
+//   Split-K: as in the main kernel, fp32 partials (no ReLU) per split, added
+//     in split order by the reduction kernel.
+//   Slot release in groups: the ring is released kGroup stages at a time
+//     (one tcgen05.commit per kGroup stages, one "empty" barrier per group)
+//     while each stage keeps its own "full" barrier, so the MMA issuer pays
+//     for fewer commits between its small MMAs.
+// Roles, barriers and bounded waits are those of gemm_kernel.cuh.
+#pragma once
+
+#include "gemm_kernel.cuh"
+
+namespace gr {
+
+template <int NP>
+struct SkinnyCfg {
+    static constexpr int kTileN = 128;                       // columns of C per tile (MMA M)
+    static constexpr int kBBytes = kTileN * kBK * 2;          // 16 KB op(B)^T tile
+    static constexpr int kABytes = NP * kBK * 2;              // NP rows of A
+    static constexpr int kStageBytes = kBBytes + kABytes;     // multiple of 1024
+    static constexpr int kGroup = 3;                          // stages released per commit
+    static constexpr int kStagesFit = (232448 - 2048) / kStageBytes;
+    static constexpr int kStagesCap = kStagesFit > 12 ? 12 : kStagesFit;
+    static constexpr int kStages = kStagesCap / kGroup * kGroup;
+    static constexpr int kGroups = kStages / kGroup;
+    static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
+    static constexpr uint32_t kTmemCols = 2 * NP < 32 ? 32 : 2 * NP;   // power of two
+};
+
+template <int NP, bool B_MN, typename OutT>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_relu_skinny_kernel(const __grid_constant__ CUtensorMap tmA,
+                            const __grid_constant__ CUtensorMap tmB, const GemmParams p)
+{
+    using Cfg = SkinnyCfg<NP>;
+    constexpr int kStages = Cfg::kStages;
+    constexpr int kGroup = Cfg::kGroup;
+    static_assert(Cfg::kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
+    static_assert(kStages % kGroup == 0 && kStages >= 2 * kGroup, "ring of whole groups");
+
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t full_bar[kStages];
+    __shared__ __align__(8) uint64_t empty_bar[Cfg::kGroups];  // one per group of stages
+    __shared__ __align__(8) uint64_t tfull_bar[2];
+    __shared__ __align__(8) uint64_t tempty_bar[2];
+    __shared__ __align__(8) uint64_t drain_bar;
+    __shared__ uint32_t tmem_slot;
+    __shared__ int abort_flag;
+
+    const int warp = static_cast<int>(threadIdx.x >> 5);
+    const int lane = static_cast<int>(threadIdx.x & 31);
+    const uint32_t tiles_base = (smem_addr(smem_raw) + 1023u) & ~1023u;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) mbar_init(smem_addr(&full_bar[s]), 1);
+        for (int gidx = 0; gidx < Cfg::kGroups; ++gidx) mbar_init(smem_addr(&empty_bar[gidx]), 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_addr(&tfull_bar[b]), 1);
+            mbar_init(smem_addr(&tempty_bar[b]), 4);
+        }
+        mbar_init(smem_addr(&drain_bar), 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensor_map(&tmA);
+        prefetch_tensor_map(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc<1>(smem_addr(&tmem_slot), Cfg::kTmemCols);
+        tmem_relinquish<1>();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem_base = tmem_slot;
+
+    const WaitCtx wc{&abort_flag, p.timeout_ns, p.sleep_ns};
+    bool aborted = false;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer (one lane)
+        if (lane == 0) {
+            const uint64_t pol_a = make_l2_policy(p.l2_a);
+            const uint64_t pol_b = make_l2_policy(p.l2_b);
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued_mask = 0, last_parity = 0;
+            for (int u = blockIdx.x; u < p.num_units && !aborted; u += gridDim.x) {
+                const WorkUnit w = decode_unit(u, p.tiles_m, p.tiles_n, p.splits, p.kblocks, p.panel);
+                const int n0 = w.n_tile * Cfg::kTileN;
+                for (int kb = w.kb0; kb < w.kb1; ++kb) {
+                    // a whole group of slots is released by one commit
+                    if (stage % kGroup == 0 &&
+                        !wait_phase_thread<false>(smem_addr(&empty_bar[stage / kGroup]), phase ^ 1u,
+                                                  wc, kErrProducer)) {
+                        aborted = true;
+                        break;
+                    }
+                    const uint32_t fb = smem_addr(&full_bar[stage]);
+                    const uint32_t b_dst = tiles_base + static_cast<uint32_t>(stage * Cfg::kStageBytes);
+                    const uint32_t a_dst = b_dst + Cfg::kBBytes;
+                    const int k0 = kb * kBK;
+                    mbar_arrive_expect_tx(fb, Cfg::kStageBytes);
+                    if constexpr (B_MN) {
+                        tma_load_2d_hint(b_dst, &tmB, fb, n0, k0, pol_b);
+                        tma_load_2d_hint(b_dst + 8192, &tmB, fb, n0 + 64, k0, pol_b);
+                    } else {
+                        tma_load_2d_hint(b_dst, &tmB, fb, k0, n0, pol_b);
+                    }
+                    tma_load_2d_hint(a_dst, &tmA, fb, k0, 0, pol_a);
+                    issued_mask |= 1u << stage;
+                    last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (aborted) {
+                for (int s = 0; s < kStages; ++s)
+                    if (issued_mask & (1u << s))
+                        if (!wait_phase_one(smem_addr(&full_bar[s]), (last_parity >> s) & 1u, 20000000ull))
+                            atomicOr(&g_gemm_device_error, kErrDrain);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer (one lane)
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int local = 0;
+            bool issued_any = false;
+            const uint64_t a_desc0 = B_MN ? smem_desc_sw128(tiles_base, 8192, 1024)
+                                          : smem_desc_sw128(tiles_base, 16, 1024);
+            const uint64_t b_desc0 = smem_desc_sw128(tiles_base + Cfg::kBBytes, 16, 1024);
+            constexpr uint64_t kAStep = B_MN ? (2048 >> 4) : (32 >> 4);
+            constexpr uint64_t kBStep = 32 >> 4;
+            constexpr uint64_t kStageStep = Cfg::kStageBytes >> 4;
+            // whether the next slot's operands were seen to have landed (peeked
+            // before the current slot's MMAs are issued)
+            bool next_ready = mbar_test_wait(smem_addr(&full_bar[0]), 0);
+            for (int u = blockIdx.x; u < p.num_units && !aborted; u += gridDim.x, ++local) {
+                const WorkUnit w = decode_unit(u, p.tiles_m, p.tiles_n, p.splits, p.kblocks, p.panel);
+                const int buf = local & 1;
+                const uint32_t tphase = static_cast<uint32_t>(local >> 1) & 1u;
+                if (!wait_phase_thread<false>(smem_addr(&tempty_bar[buf]), tphase ^ 1u, wc,
+                                              kErrMmaAccum)) {
+                    aborted = true;
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * NP);
+                for (int kb = w.kb0; kb < w.kb1; ++kb) {
+                    if (!next_ready &&
+                        !wait_phase_thread<false>(smem_addr(&full_bar[stage]), phase, wc,
+                                                  kErrMmaOperands)) {
+                        aborted = true;
+                        break;
+                    }
+                    const int next_stage = stage + 1 == kStages ? 0 : stage + 1;
+                    const uint32_t next_phase = next_stage == 0 ? phase ^ 1u : phase;
+                    next_ready = mbar_test_wait(smem_addr(&full_bar[next_stage]), next_phase);
+                    const uint64_t so = static_cast<uint64_t>(stage) * kStageStep;
+#pragma unroll
+                    for (int k = 0; k < kBK / 16; ++k)
+                        umma_f16<1>(d_tmem, a_desc0 + so + k * kAStep, b_desc0 + so + k * kBStep,
+                                    p.idesc, (kb > w.kb0 || k > 0) ? 1u : 0u);
+                    if (stage % kGroup == kGroup - 1) umma_commit(smem_addr(&empty_bar[stage / kGroup]));
+                    issued_any = true;
+                    stage = next_stage;
+                    phase = next_phase;
+                }
+                if (aborted) break;
+                umma_commit(smem_addr(&tfull_bar[buf]));
+            }
+            if (aborted && issued_any) {
+                umma_commit(smem_addr(&drain_bar));
+                if (!wait_phase_one(smem_addr(&drain_bar), 0, 20000000ull))
+                    atomicOr(&g_gemm_device_error, kErrDrain);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------ epilogue (warps 2..5)
+        const int q = warp & 3;
+        int local = 0;
+        for (int u = blockIdx.x; u < p.num_units && !aborted; u += gridDim.x, ++local) {
+            const WorkUnit w = decode_unit(u, p.tiles_m, p.tiles_n, p.splits, p.kblocks, p.panel);
+            const int buf = local & 1;
+            const uint32_t tphase = static_cast<uint32_t>(local >> 1) & 1u;
+            if (!wait_phase<false>(smem_addr(&tfull_bar[buf]), tphase, wc, kErrEpilogue)) {
+                aborted = true;
+                break;
+            }
+            tc_fence_after_sync();
+            const int n = w.n_tile * Cfg::kTileN + q * 32 + lane;   // column of C
+            const bool n_ok = n < p.N;
+            OutT *out = reinterpret_cast<OutT *>(p.C) + static_cast<int64_t>(w.split) * p.split_stride;
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                   static_cast<uint32_t>(buf * NP);
+#pragma unroll 1
+            for (int c = 0; c < NP; c += 16) {
+                if (c >= p.M) break;  // warp-uniform
+                uint32_t v[16];
+                tmem_load_16cols(taddr + static_cast<uint32_t>(c), v);
+                tmem_load_wait();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int m = c + i;
+                    if (n_ok && m < p.M) {
+                        float x = __uint_as_float(v[i]);
+                        if (p.relu) x = fmaxf(x, 0.0f);
+                        out[static_cast<int64_t>(m) * p.ldc + n] = convert_out<OutT>(x);
+                    }
+                }
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_local(smem_addr(&tempty_bar[buf]));
+        }
+    }
+
+    __syncwarp();
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc<1>(tmem_base, Cfg::kTmemCols);
+    }
+}
+
+}  // namespace gr
