@@ -114,7 +114,8 @@ struct WorkUnit {
 
 // Unit -> (tile, split).  Splits of one tile are adjacent; tiles are walked
 // panel by panel (`panel` tile rows per panel, all tile columns), column-major
-// inside a panel.
+// inside a panel, and every other panel walks its columns backwards so the
+// first tiles of a panel reuse the B columns the previous panel read last.
 __host__ __device__ __forceinline__ WorkUnit decode_unit(int u, int tiles_m, int tiles_n,
                                                          int splits, int kblocks, int panel)
 {
@@ -128,9 +129,19 @@ __host__ __device__ __forceinline__ WorkUnit decode_unit(int u, int tiles_m, int
     const int rows_here = panel < left ? panel : left;
     w.m_tile = pi * panel + r % rows_here;
     w.n_tile = r / rows_here;
+    if (pi & 1) w.n_tile = tiles_n - 1 - w.n_tile;
     w.kb0 = static_cast<int>(static_cast<int64_t>(w.split) * kblocks / splits);
     w.kb1 = static_cast<int>(static_cast<int64_t>(w.split + 1) * kblocks / splits);
     return w;
+}
+
+// The i-th K block a CTA processes for its `local`-th unit.  Consecutive
+// units of a CTA alternate the direction of the K loop: at a wave boundary
+// the next tiles start on the K range whose A rows (same panel) were read
+// most recently and are still in L2.  The sum order changes, nothing else.
+__device__ __forceinline__ int k_block_at(const WorkUnit &w, int i, int local)
+{
+    return (local & 1) ? w.kb1 - 1 - i : w.kb0 + i;
 }
 
 struct WaitCtx {
@@ -343,11 +354,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t phase = 0;
             uint32_t issued_mask = 0;  // stages that received at least one load
             uint32_t last_parity = 0;  // parity of the last phase issued per stage (bit s)
-            for (int u = cluster_id; u < p.num_units && !aborted; u += num_clusters) {
+            int local = 0;
+            for (int u = cluster_id; u < p.num_units && !aborted; u += num_clusters, ++local) {
                 const WorkUnit w = decode_unit(u, p.tiles_m, p.tiles_n, p.splits, p.kblocks, p.panel);
                 const int m_row = w.m_tile * Cfg::kTileM + static_cast<int>(rank) * kBM;
                 const int n_col = w.n_tile * kBN + static_cast<int>(rank) * Cfg::kBNCta;
-                for (int kb = w.kb0; kb < w.kb1; ++kb) {
+                // K direction alternates per unit (see k_block_at)
+                for (int i = 0; i < w.kb1 - w.kb0; ++i) {
+                    const int kb = k_block_at(w, i, local);
                     // the slot is released by the MMA's tcgen05.commit (local in both CTAs)
                     if (!wait_phase_thread<false>(smem_addr(&empty_bar[stage]), phase ^ 1u, wc,
                                                   kErrProducer)) {
@@ -442,7 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tc_fence_after_sync();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * kBN);
-                for (int kb = w.kb0; kb < w.kb1; ++kb) {
+                for (int i = 0; i < w.kb1 - w.kb0; ++i) {
                     if (!next_ready &&
                         !wait_phase_thread<false>(smem_addr(&full_bar[stage]), phase, wc,
                                                   kErrMmaOperands)) {
@@ -459,7 +473,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint64_t kin = static_cast<uint64_t>(k % (kBK / 16));
                         umma_f16<CG>(d_tmem, a_desc0 + so + sub * kASubStep + kin * kAStep,
                                      b_desc0 + so + sub * kBSubStep + kin * kBStep, p.idesc,
-                                     (kb > w.kb0 || k > 0) ? 1u : 0u);
+                                     (i > 0 || k > 0) ? 1u : 0u);
                     }
                     if constexpr (PAIR)
                         umma_commit_pair(smem_addr(&empty_bar[stage]), 0x3);
