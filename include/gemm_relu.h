@@ -92,6 +92,8 @@ typedef struct {
                             the hardware default                                        */
     int swap_ab;         /* skinny-M kernel computing C^T = op(B)^T A^T: 0 = auto (M <= 64
                             and cta_pair auto), 1 = use it (needs M <= 128), 2 = never     */
+    int stream_k;        /* skinny kernel: 1 = spread the K blocks of all column tiles
+                            evenly over the CTAs (stream-K) instead of split-K; 0 = off  */
 } gemm_relu_options_t;
 /* cta_pair: 0 = auto, 1 = force the 2-CTA (256 x 256 tile, cta_group::2)
  * kernel, 2 = force the 1-CTA (128 x 256 tile) kernel.  Split-K always uses
@@ -113,6 +115,9 @@ typedef struct {
     int stages;          /* shared-memory pipeline depth                                  */
     int pack_a, pack_b;  /* 1 = operand is re-pitched into the workspace first            */
     int swap_ab;         /* 1 = skinny-M kernel: tiles of tile_n columns of C, all M rows  */
+    int stream_k;        /* skinny kernel only: > 0 = the tiles_n * kblocks K blocks are
+                            spread over this many CTAs (stream-K); 0 = whole tiles        */
+    int sk_max_seg;      /* stream-K: partial-sum slots per tile                            */
     int64_t workspace_bytes;
 } gemm_relu_plan_t;
 
@@ -147,11 +152,20 @@ typedef struct {
     int tile_row, tile_col, kb_begin, kb_end, split;
 } gemm_relu_unit_t;
 
-/* The unit the persistent kernels process as number `u` (0 <= u < units):
+/* The unit the persistent kernels process as number `u` (0 <= u < units) of a
+ * plan without stream-K (stream-K plans: see gemm_relu_plan_segments):
  * the same tile walk the device uses (panels of `panel` tile rows, column by
  * column inside a panel, splits of one tile adjacent).  Host only. */
 GEMM_RELU_API gemm_status_t gemm_relu_plan_unit(const gemm_relu_plan_t *plan, int u,
                                                 gemm_relu_unit_t *unit);
+
+/* Stream-K plans (plan->stream_k > 0): the pieces CTA `cta` processes, in
+ * order, written to out[0 .. max) (tile_row = 0, tile_col = column tile,
+ * K blocks [kb_begin, kb_end), split = partial-sum slot within the tile or
+ * -1 when the CTA owns the whole tile).  Returns the number of pieces (may
+ * exceed max; only max are written) or -1 on bad arguments.  Host only. */
+GEMM_RELU_API int gemm_relu_plan_segments(const gemm_relu_plan_t *plan, int cta,
+                                          gemm_relu_unit_t *out, int max);
 
 /* Static description of a status code (never NULL). */
 GEMM_RELU_API const char *gemm_relu_status_string(gemm_status_t status);

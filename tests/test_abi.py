@@ -75,12 +75,17 @@ def test_plans_for_the_workloads(lib):
 
     p = plan(wl.WORKLOADS["skinny64x8192x8192_f16"])
     assert p["swap_ab"] == 1 and p["tile_m"] == 64 and p["tile_n"] == 128
-    assert p["tiles_n"] == 64 and p["split_k"] == 2 and p["units"] == 128
+    assert p["tiles_n"] == 64 and p["split_k"] == 2 and p["units"] == 128 and p["stream_k"] == 0
     assert p["workspace_bytes"] >= 2 * 64 * 8192 * 4
 
     p = plan(wl.WORKLOADS["skinny16x16384x4096_f16"])
     assert p["swap_ab"] == 1 and p["tile_m"] == 16 and p["split_k"] == 1 and p["units"] == 128
     assert p["workspace_bytes"] == 0
+
+    p = plan(wl.WORKLOADS["skinny64x8192x8192_f16"], stream_k=1)
+    assert p["stream_k"] == 148 and p["grid_ctas"] == 148
+    assert p["sk_max_seg"] == 4                        # 8192 blocks / 148 CTAs >= 55 each
+    assert p["workspace_bytes"] >= 64 * 4 * 64 * 128 * 4
     # the main kernel's split-K path for the same shape when swap-AB is off
     p = plan(wl.WORKLOADS["skinny64x8192x8192_f16"], swap_ab=2)
     assert p["swap_ab"] == 0 and p["cta_pair"] == 0 and p["split_k"] == 4
@@ -107,6 +112,39 @@ def test_options_override_the_plan(lib):
         plan(w, stage_k=96)
 
 
+@pytest.mark.parametrize("M,N,K,opt", [
+    (64, 8192, 8192, {}),
+    (16, 16384, 4096, {}),
+    (100, 1000, 3000, {"swap_ab": 1, "split_k": 5}),
+    (1, 300, 520, {"max_ctas": 7}),
+    (33, 40000, 1024, {}),
+])
+def test_stream_k_covers_every_k_block_once(lib, M, N, K, opt):
+    p = g.gemm_relu_plan(M, N, K, torch.float16, torch.float16, False,
+                         options={**opt, "stream_k": 1})
+    assert p["swap_ab"] == 1 and p["stream_k"] > 0
+    seen = {}
+    for cta in range(p["stream_k"]):
+        segs = g.gemm_relu_plan_segments(p, cta)
+        assert segs, "every CTA has work"
+        for tile, kb0, kb1, slot in segs:
+            assert 0 <= tile < p["tiles_n"] and 0 <= kb0 < kb1 <= p["kblocks"]
+            assert slot == -1 or 0 <= slot < p["sk_max_seg"]
+            seen.setdefault(tile, []).append((kb0, kb1, slot))
+    assert sorted(seen) == list(range(p["tiles_n"]))
+    for pieces in seen.values():
+        pieces.sort()
+        assert pieces[0][0] == 0 and pieces[-1][1] == p["kblocks"]
+        assert all(a[1] == b[0] for a, b in zip(pieces, pieces[1:]))
+        slots = [s for _, _, s in pieces]
+        if len(pieces) == 1:
+            assert slots == [-1]                      # owned whole: written directly
+        else:
+            assert slots == list(range(len(pieces)))  # the fix-up adds slots 0.. in order
+    with pytest.raises(g.GemmError):
+        g.gemm_relu_plan_unit(p, 0)
+
+
 @pytest.mark.parametrize("M,np_", [(1, 16), (16, 16), (17, 32), (32, 32), (33, 64), (64, 64),
                                     (65, 128), (128, 128)])
 def test_swap_ab_bucket(lib, M, np_):
@@ -129,11 +167,12 @@ def test_misaligned_base_pointer_is_repitched(lib):
 @pytest.mark.parametrize("M,N,K,opt", [
     (8192, 8192, 8192, {}),
     (5000, 3001, 2050, {}),
-    (64, 8192, 8192, {}),
+    (64, 8192, 8192, {"swap_ab": 2}),
     (300, 700, 1000, {"split_k": 7, "panel": 3}),
     (1000, 300, 130, {"cta_pair": g.GEMM_CTA_SINGLE, "panel": 5}),
     (257, 257, 65, {"panel": 1}),
     (600, 300, 1000, {"stage_k": 64}),
+    (100, 1000, 3000, {"swap_ab": 1, "split_k": 1}),
     (64, 8192, 8192, {"swap_ab": 1}),
     (100, 1000, 3000, {"swap_ab": 1, "split_k": 5}),
 ])

@@ -101,6 +101,8 @@ VARIANTS = {
     "l2_hints": {"l2_hint_a": 2, "l2_hint_b": 1, "c_streaming": 1, "wait_sleep_ns": 20000},
     "swap": {"swap_ab": 1},
     "swap_split3": {"swap_ab": 1, "split_k": 3},
+    "swap_streamk": {"swap_ab": 1, "stream_k": 1},
+    "swap_streamk_few": {"swap_ab": 1, "stream_k": 1, "max_ctas": 7},
     "no_swap": {"swap_ab": 2},
 }
 
@@ -122,7 +124,8 @@ def test_dtypes_and_relu(in_dtype, out_dtype, trans_b, relu, variant):
               dist="normal")
 
 
-@pytest.mark.parametrize("variant", ["swap", "swap_split3", "auto", "no_swap"])
+@pytest.mark.parametrize("variant", ["swap", "swap_split3", "swap_streamk", "swap_streamk_few",
+                                     "auto", "no_swap"])
 @pytest.mark.parametrize("trans_b", [False, True])
 @pytest.mark.parametrize("M", [1, 7, 16, 17, 33, 64, 65, 100, 128])
 def test_skinny_M(M, trans_b, variant):
@@ -136,6 +139,8 @@ def test_skinny_dtypes(in_dtype, out_dtype, relu):
     full_case(40, 777, 520, in_dtype, out_dtype, True, relu, VARIANTS["swap"], seed=3,
               dist="normal")
     full_case(40, 776, 520, in_dtype, out_dtype, False, relu, VARIANTS["swap_split3"], seed=4,
+              dist="normal")
+    full_case(40, 777, 1520, in_dtype, out_dtype, True, relu, VARIANTS["swap_streamk"], seed=5,
               dist="normal")
 
 

@@ -35,7 +35,7 @@ EXPORTS = (
     "gemm_relu", "gemm_relu_ex", "gemm_relu_plan", "gemm_relu_status_string",
     "gemm_relu_last_cuda_error", "gemm_relu_last_device_error", "gemm_relu_selftest_timeout",
     "gemm_relu_release_workspace", "gemm_relu_version", "gemm_relu_plan_unit",
-    "gemm_relu_splitk_noalloc",
+    "gemm_relu_splitk_noalloc", "gemm_relu_plan_segments",
 )
 
 # size of the static device array behind gemm_relu_splitk_noalloc (header constant)
@@ -58,13 +58,15 @@ class GemmOptions(ctypes.Structure):
         ("c_streaming", ctypes.c_int),
         ("wait_sleep_ns", ctypes.c_uint32),
         ("swap_ab", ctypes.c_int),
+        ("stream_k", ctypes.c_int),
     ]
 
 
 class GemmPlan(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "cta_pair", "tile_m", "tile_n", "tile_k", "tiles_m", "tiles_n", "kblocks", "split_k",
-        "panel", "units", "grid_ctas", "stages", "pack_a", "pack_b", "swap_ab")] + [
+        "panel", "units", "grid_ctas", "stages", "pack_a", "pack_b", "swap_ab", "stream_k",
+        "sk_max_seg")] + [
         ("workspace_bytes", ctypes.c_int64)]
 
     def as_dict(self) -> dict:
@@ -104,6 +106,9 @@ def load():
                                            ctypes.POINTER(GemmOptions), ctypes.POINTER(GemmPlan)]
             lib.gemm_relu_plan_unit.argtypes = [ctypes.POINTER(GemmPlan), i32,
                                                 ctypes.POINTER(GemmUnit)]
+            lib.gemm_relu_plan_segments.argtypes = [ctypes.POINTER(GemmPlan), i32,
+                                                    ctypes.POINTER(GemmUnit), i32]
+            lib.gemm_relu_plan_segments.restype = i32
             lib.gemm_relu_status_string.argtypes = [i32]
             lib.gemm_relu_status_string.restype = ctypes.c_char_p
             lib.gemm_relu_last_cuda_error.argtypes = []
@@ -213,6 +218,19 @@ def gemm_relu_plan_unit(plan: dict, u: int) -> tuple[int, int, int, int, int]:
     unit = GemmUnit()
     _check(load().gemm_relu_plan_unit(ctypes.byref(p), int(u), ctypes.byref(unit)))
     return unit.tile_row, unit.tile_col, unit.kb_begin, unit.kb_end, unit.split
+
+
+def gemm_relu_plan_segments(plan: dict, cta: int) -> list[tuple[int, int, int, int]]:
+    """Stream-K plans: [(tile_col, kb_begin, kb_end, slot or -1)] processed by CTA `cta`."""
+    p = GemmPlan(**{k: plan[k] for k, _ in GemmPlan._fields_})
+    buf = (GemmUnit * 64)()
+    n = load().gemm_relu_plan_segments(ctypes.byref(p), int(cta), buf, 64)
+    if n < 0:
+        raise GemmError(GEMM_ERR_INVALID_ARG, "not a stream-K plan or bad CTA index")
+    if n > 64:
+        buf = (GemmUnit * n)()
+        n = load().gemm_relu_plan_segments(ctypes.byref(p), int(cta), buf, n)
+    return [(buf[i].tile_col, buf[i].kb_begin, buf[i].kb_end, buf[i].split) for i in range(n)]
 
 
 def gemm_relu_status_string(status: int) -> str:

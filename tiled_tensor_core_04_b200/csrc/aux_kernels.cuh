@@ -54,18 +54,70 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const float *__restr
     }
 }
 
+// Stream-K fix-up for the skinny kernel: for every column tile split between
+// CTAs, C[m, n] = relu(sum of its pieces' partials, in slot order), cast.
+// Tiles owned whole by one CTA were written by the GEMM kernel and are skipped.
+template <typename OutT>
+__global__ void __launch_bounds__(256) streamk_reduce_kernel(const float *__restrict__ ws,
+                                                             OutT *__restrict__ C, int M, int N,
+                                                             int64_t ldc, int tiles, int kblocks,
+                                                             int64_t T, int G, int max_seg, int relu)
+{
+    constexpr int kTileN = 128;
+    const int64_t per_tile = static_cast<int64_t>(M) * kTileN;
+    const int64_t total = per_tile * tiles;
+    for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int tile = static_cast<int>(idx / per_tile);
+        const int64_t r = idx - static_cast<int64_t>(tile) * per_tile;
+        const int m = static_cast<int>(r / kTileN);
+        const int nl = static_cast<int>(r - static_cast<int64_t>(m) * kTileN);
+        const int n = tile * kTileN + nl;
+        if (n >= N) continue;
+        const int first = sk_owner(static_cast<int64_t>(tile) * kblocks, T, G);
+        const int last = sk_owner(static_cast<int64_t>(tile + 1) * kblocks - 1, T, G);
+        if (last == first) continue;  // written whole by its owner
+        const float *src = ws + static_cast<int64_t>(tile) * max_seg * per_tile + r;
+        float acc = src[0];
+        for (int s = 1; s <= last - first; ++s) acc += src[static_cast<int64_t>(s) * per_tile];
+        if (relu) acc = fmaxf(acc, 0.0f);
+        C[static_cast<int64_t>(m) * ldc + n] = convert_out<OutT>(acc);
+    }
+}
+
 // dst[r * dst_pitch + c] = src[r * cols + c] for r < rows, c < cols (16-bit).
+// dst is 16-byte aligned with a pitch of a multiple of 8 elements; src rows
+// may start on any 2-byte boundary.  One warp copies a row at a time, lane l
+// taking 8-element chunks l, l + 32, ...: 16-byte stores, and 4-byte loads
+// where the source row is 4-byte aligned (2-byte loads otherwise).
 __global__ void __launch_bounds__(256) repitch_kernel(const uint16_t *__restrict__ src,
                                                       int64_t rows, int64_t cols,
                                                       uint16_t *__restrict__ dst,
                                                       int64_t dst_pitch)
 {
-    for (int64_t r = blockIdx.y; r < rows; r += gridDim.y) {
-        const uint16_t *s = src + r * cols;
-        uint16_t *d = dst + r * dst_pitch;
-        for (int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c < cols;
-             c += static_cast<int64_t>(gridDim.x) * blockDim.x)
-            d[c] = s[c];
+    const int lane = static_cast<int>(threadIdx.x & 31);
+    const int64_t warp0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    const int64_t chunks = cols / 8;
+    for (int64_t r = warp0; r < rows; r += nwarps) {
+        const uint16_t *srow = src + r * cols;
+        uint16_t *drow = dst + r * dst_pitch;
+        if ((reinterpret_cast<uintptr_t>(srow) & 3u) == 0) {
+            for (int64_t c = lane; c < chunks; c += 32) {
+                const uint32_t *s4 = reinterpret_cast<const uint32_t *>(srow + c * 8);
+                *reinterpret_cast<uint4 *>(drow + c * 8) = make_uint4(s4[0], s4[1], s4[2], s4[3]);
+            }
+        } else {
+            for (int64_t c = lane; c < chunks; c += 32) {
+                const uint16_t *s2 = srow + c * 8;
+                uint32_t w[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    w[i] = static_cast<uint32_t>(s2[2 * i]) | (static_cast<uint32_t>(s2[2 * i + 1]) << 16);
+                *reinterpret_cast<uint4 *>(drow + c * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        }
+        for (int64_t e = chunks * 8 + lane; e < cols; e += 32) drow[e] = srow[e];
     }
 }
 

@@ -78,7 +78,30 @@ struct GemmParams {
     int l2_a, l2_b;        // L2 eviction priority of the A / B loads (0 normal, 1 first, 2 last)
     int c_stream;          // 1: store C with evict-first (streaming) stores
     uint32_t sleep_ns;     // suspend-time hint for the epilogue's accumulator waits
+    // stream-K (skinny kernel): sk_iters > 0 spreads tiles_n * kblocks K blocks
+    // evenly over the CTAs; tiles split between CTAs leave fp32 partials in
+    // sk_ws, slot (tile * sk_max_seg + segment), each M x 128, row pitch 128
+    int64_t sk_iters;
+    int sk_max_seg;
+    float *sk_ws;
 };
+
+// ------------------------------------------------------------------ stream-K
+// CTA c of G owns K-block iterations [sk_begin(c), sk_begin(c + 1)) of the
+// T = tiles * kblocks iterations, tile-major.
+__host__ __device__ __forceinline__ int64_t sk_begin(int64_t c, int64_t T, int64_t G)
+{
+    return c * T / G;
+}
+
+// The CTA whose range contains iteration x.
+__host__ __device__ __forceinline__ int sk_owner(int64_t x, int64_t T, int64_t G)
+{
+    int64_t c = (x * G) / T;
+    while (c + 1 < G && sk_begin(c + 1, T, G) <= x) ++c;
+    while (c > 0 && sk_begin(c, T, G) > x) --c;
+    return static_cast<int>(c);
+}
 
 constexpr int kThreads = 192;  // 6 warps
 constexpr int kBM = 128;       // rows of A per CTA

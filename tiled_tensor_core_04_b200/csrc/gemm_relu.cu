@@ -244,7 +244,8 @@ gemm_status_t make_plan(int64_t M, int64_t N, int64_t K, gemm_dtype_t in, gemm_d
     if (opts) o = *opts;
     if (o.cta_pair < 0 || o.cta_pair > 2 || o.split_k < 0 || o.panel < 0 || o.max_ctas < 0 ||
         (o.stage_k != 0 && o.stage_k != 64 && o.stage_k != 128) || o.l2_hint_a < 0 ||
-        o.l2_hint_a > 2 || o.l2_hint_b < 0 || o.l2_hint_b > 2 || o.c_streaming < 0 || o.c_streaming > 1 || o.swap_ab < 0 || o.swap_ab > 2)
+        o.l2_hint_a > 2 || o.l2_hint_b < 0 || o.l2_hint_b > 2 || o.c_streaming < 0 || o.c_streaming > 1 || o.swap_ab < 0 || o.swap_ab > 2 ||
+        o.stream_k < 0 || o.stream_k > 1)
         return GEMM_ERR_INVALID_ARG;
 
     gemm_relu_plan_t p = {};
@@ -265,25 +266,42 @@ gemm_status_t make_plan(int64_t M, int64_t N, int64_t K, gemm_dtype_t in, gemm_d
         p.tile_k = kBK;
         p.tiles_m = 1;
         p.tiles_n = static_cast<int>(ceil_div(N, 128));
-        int64_t sp = o.split_k;
-        if (sp == 0) {
-            sp = 1;
-            if (p.tiles_n * 2 <= num_sms && p.kblocks >= 8) {
-                sp = std::max<int64_t>(1, num_sms / p.tiles_n);
-                sp = std::min<int64_t>(sp, p.kblocks / 4);
-                sp = std::min<int64_t>(sp, 32);
-            }
-        }
-        sp = p.kblocks > 0 ? std::max<int64_t>(1, std::min<int64_t>(sp, p.kblocks)) : 1;
-        const int64_t su = static_cast<int64_t>(p.tiles_n) * sp;
-        if (su > INT32_MAX) return GEMM_ERR_INVALID_ARG;
-        p.split_k = static_cast<int>(sp);
-        p.panel = 1;
-        p.units = static_cast<int>(su);
-        p.stages = skinny_stages(np);
+        // K split in equal ranges when whole column tiles cannot fill the SMs
+        // (CTAs walk K in step); stream-K (an even spread of the tiles_n *
+        // kblocks K blocks over the CTAs) only when asked for.
         int64_t ctas = num_sms;
         if (o.max_ctas > 0) ctas = std::min<int64_t>(ctas, o.max_ctas);
-        p.grid_ctas = static_cast<int>(std::min<int64_t>(su, ctas));
+        const int64_t T = static_cast<int64_t>(p.tiles_n) * p.kblocks;
+        p.stream_k = 0;
+        if (o.stream_k == 1 && T >= 1) {
+            int64_t G = std::min<int64_t>(ctas, T);
+            if (o.split_k >= 2) G = std::min<int64_t>(G, static_cast<int64_t>(p.tiles_n) * o.split_k);
+            p.stream_k = static_cast<int>(G);
+            p.split_k = 1;
+            p.units = static_cast<int>(G);
+            p.grid_ctas = static_cast<int>(G);
+            const int64_t per = T / G;  // every CTA owns >= per K blocks
+            p.sk_max_seg = static_cast<int>((p.kblocks + per - 1) / per + 1);
+        } else {
+            int64_t sp = o.split_k;
+            if (sp == 0) {
+                // too few column tiles to fill the SMs: split K, >= 4 K blocks each
+                sp = 1;
+                if (static_cast<int64_t>(p.tiles_n) * 2 <= ctas && p.kblocks >= 8) {
+                    sp = std::max<int64_t>(1, ctas / p.tiles_n);
+                    sp = std::min<int64_t>(sp, p.kblocks / 4);
+                    sp = std::min<int64_t>(sp, 32);
+                }
+            }
+            sp = p.kblocks > 0 ? std::max<int64_t>(1, std::min<int64_t>(sp, p.kblocks)) : 1;
+            const int64_t su = static_cast<int64_t>(p.tiles_n) * sp;
+            if (su > INT32_MAX) return GEMM_ERR_INVALID_ARG;
+            p.split_k = static_cast<int>(sp);
+            p.units = static_cast<int>(su);
+            p.grid_ctas = static_cast<int>(std::min<int64_t>(su, ctas));
+        }
+        p.panel = 1;
+        p.stages = skinny_stages(np);
     }
 
     int64_t split = o.split_k;
@@ -359,6 +377,9 @@ gemm_status_t make_plan(int64_t M, int64_t N, int64_t K, gemm_dtype_t in, gemm_d
     if (p.split_k > 1) {
         l.split_off = off;
         off = round_up(off + static_cast<int64_t>(p.split_k) * M * N * 4, 256);
+    } else if (p.stream_k > 0) {
+        l.split_off = off;
+        off = round_up(off + static_cast<int64_t>(p.tiles_n) * p.sk_max_seg * M * 128 * 4, 256);
     }
     l.total = off;
     p.workspace_bytes = off;
@@ -424,11 +445,50 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
+// Recently encoded maps, per host thread (encoding is pure host work, but it
+// is the largest part of a small call's host time).
+struct MapKey {
+    const void *base;
+    int64_t inner, outer, pitch;
+    int dt, box_inner, box_outer;
+    bool operator==(const MapKey &o) const
+    {
+        return base == o.base && inner == o.inner && outer == o.outer && pitch == o.pitch &&
+               dt == o.dt && box_inner == o.box_inner && box_outer == o.box_outer;
+    }
+};
+constexpr int kMapCache = 16;
+thread_local MapKey t_map_keys[kMapCache];
+thread_local CUtensorMap t_maps[kMapCache];
+thread_local int t_map_used = 0, t_map_next = 0;
+
+gemm_status_t encode_2d_uncached(CUtensorMap *map, const void *base, gemm_dtype_t dt, int64_t inner,
+                                 int64_t outer, int64_t pitch_elems, int box_inner, int box_outer);
+
 // 2-D map over a row-major 16-bit matrix: inner extent `inner` (contiguous),
 // `outer` rows `pitch_elems` apart, box {box_inner, box_outer}, 128-byte swizzle,
 // out-of-range elements read as zero.
 gemm_status_t encode_2d(CUtensorMap *map, const void *base, gemm_dtype_t dt, int64_t inner,
                         int64_t outer, int64_t pitch_elems, int box_inner, int box_outer)
+{
+    const MapKey key{base, inner, outer, pitch_elems, static_cast<int>(dt), box_inner, box_outer};
+    for (int i = 0; i < t_map_used; ++i)
+        if (t_map_keys[i] == key) {
+            *map = t_maps[i];
+            return GEMM_OK;
+        }
+    gemm_status_t st = encode_2d_uncached(map, base, dt, inner, outer, pitch_elems, box_inner, box_outer);
+    if (st != GEMM_OK) return st;
+    const int slot = t_map_next;
+    t_map_keys[slot] = key;
+    t_maps[slot] = *map;
+    t_map_next = (t_map_next + 1) % kMapCache;
+    if (t_map_used < kMapCache) ++t_map_used;
+    return GEMM_OK;
+}
+
+gemm_status_t encode_2d_uncached(CUtensorMap *map, const void *base, gemm_dtype_t dt, int64_t inner,
+                                 int64_t outer, int64_t pitch_elems, int box_inner, int box_outer)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn) {
@@ -463,11 +523,13 @@ uint32_t make_idesc(gemm_dtype_t in, bool b_mn, int mma_m, int mma_n, bool a_mn 
 gemm_status_t launch_repitch(const void *src, int64_t rows, int64_t cols, void *dst,
                              int64_t pitch, cudaStream_t stream)
 {
-    dim3 block(256);
-    dim3 grid(static_cast<unsigned>(std::min<int64_t>(ceil_div(cols, 256), 64)),
-              static_cast<unsigned>(std::min<int64_t>(rows, 65535)));
-    repitch_kernel<<<grid, block, 0, stream>>>(static_cast<const uint16_t *>(src), rows, cols,
-                                                static_cast<uint16_t *>(dst), pitch);
+    // one warp per row at a time, at most 8 blocks of 8 warps per SM
+    int sms = 148;
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(ceil_div(rows, 8), 8LL * sms));
+    repitch_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
+        static_cast<const uint16_t *>(src), rows, cols, static_cast<uint16_t *>(dst), pitch);
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? GEMM_OK : cuda_fail(e, "repitch launch");
 }
@@ -498,10 +560,10 @@ gemm_status_t launch_skinny(const gemm_relu_plan_t &plan, const void *a_src, int
         st = encode_2d(&tmB, b_src, in, K, N, b_pitch, kBK, 128);
     if (st != GEMM_OK) return st;
 
+    const bool sk = plan.stream_k > 0;
     const bool split = plan.split_k > 1;
-    const gemm_dtype_t kout = split ? GEMM_F32 : out;
     GemmParams p = {};
-    p.C = split ? split_ws : C;
+    p.C = C;
     p.ldc = N;
     p.split_stride = split ? M * N : 0;
     p.M = static_cast<int>(M);
@@ -513,7 +575,7 @@ gemm_status_t launch_skinny(const gemm_relu_plan_t &plan, const void *a_src, int
     p.kblocks = plan.kblocks;
     p.panel = plan.panel;
     p.num_units = plan.units;
-    p.relu = split ? 0 : (relu ? 1 : 0);
+    p.relu = relu ? 1 : 0;
     p.vec_ok = 0;
     // MMA: 128 columns of C (op(B)^T, MN-major when B is stored (K, N)) x np rows of C
     p.idesc = make_idesc(in, false, 128, np, b_mn);
@@ -521,9 +583,12 @@ gemm_status_t launch_skinny(const gemm_relu_plan_t &plan, const void *a_src, int
     p.l2_a = opts ? opts->l2_hint_a : 0;
     p.l2_b = opts ? opts->l2_hint_b : 0;
     p.sleep_ns = (opts && opts->wait_sleep_ns) ? opts->wait_sleep_ns : 0;
+    p.sk_iters = sk ? static_cast<int64_t>(plan.tiles_n) * plan.kblocks : 0;
+    p.sk_max_seg = sk ? plan.sk_max_seg : 0;
+    p.sk_ws = (sk || split) ? static_cast<float *>(split_ws) : nullptr;
     {
         std::lock_guard<std::mutex> lock(g_dev_mutex);
-        st = ensure_skinny_attr(*dev, np, b_mn, kout);
+        st = ensure_skinny_attr(*dev, np, b_mn, out);
     }
     if (st != GEMM_OK) return st;
     cudaLaunchConfig_t cfg = {};
@@ -532,9 +597,23 @@ gemm_status_t launch_skinny(const gemm_relu_plan_t &plan, const void *a_src, int
     cfg.dynamicSmemBytes = skinny_smem(np);
     cfg.stream = stream;
     cfg.numAttrs = 0;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, pick_skinny(np, b_mn, kout), tmA, tmB, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, pick_skinny(np, b_mn, out), tmA, tmB, p);
     if (e != cudaSuccess) return cuda_fail(e, "skinny gemm kernel launch");
-    if (split) {
+    if (sk) {
+        const int64_t total = static_cast<int64_t>(plan.tiles_n) * M * 128;
+        const int grid = static_cast<int>(std::min<int64_t>(ceil_div(total, 256),
+                                                            static_cast<int64_t>(dev->sms) * 8));
+        const float *wsf = static_cast<const float *>(split_ws);
+        const int64_t T = p.sk_iters;
+        const int G = plan.stream_k;
+        switch (out) {
+        case GEMM_F16: streamk_reduce_kernel<__half><<<grid, 256, 0, stream>>>(wsf, static_cast<__half *>(C), p.M, p.N, N, plan.tiles_n, plan.kblocks, T, G, plan.sk_max_seg, p.relu); break;
+        case GEMM_BF16: streamk_reduce_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(wsf, static_cast<__nv_bfloat16 *>(C), p.M, p.N, N, plan.tiles_n, plan.kblocks, T, G, plan.sk_max_seg, p.relu); break;
+        default: streamk_reduce_kernel<float><<<grid, 256, 0, stream>>>(wsf, static_cast<float *>(C), p.M, p.N, N, plan.tiles_n, plan.kblocks, T, G, plan.sk_max_seg, p.relu); break;
+        }
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "stream-K fix-up launch");
+    } else if (split) {
         const int64_t n_total = M * N;
         const int vec4 = (n_total % 4) == 0 ? 1 : 0;
         const int grid = static_cast<int>(std::min<int64_t>(ceil_div(n_total / (vec4 ? 4 : 1), 256),
@@ -707,9 +786,39 @@ gemm_status_t gemm_relu_plan(int64_t M, int64_t N, int64_t K, gemm_dtype_t in_dt
                      plan, nullptr);
 }
 
+int gemm_relu_plan_segments(const gemm_relu_plan_t *plan, int cta, gemm_relu_unit_t *out, int max)
+{
+    if (!plan || plan->stream_k <= 0 || cta < 0 || cta >= plan->stream_k || max < 0 ||
+        (max > 0 && !out) || plan->kblocks <= 0)
+        return -1;
+    const int64_t T = static_cast<int64_t>(plan->tiles_n) * plan->kblocks;
+    const int64_t G = plan->stream_k;
+    int64_t it = sk_begin(cta, T, G);
+    const int64_t end = sk_begin(cta + 1, T, G);
+    int n = 0;
+    while (it < end) {
+        const int tile = static_cast<int>(it / plan->kblocks);
+        const int kb0 = static_cast<int>(it - static_cast<int64_t>(tile) * plan->kblocks);
+        const int kb1 = static_cast<int>(std::min<int64_t>(plan->kblocks, kb0 + (end - it)));
+        const int first = sk_owner(static_cast<int64_t>(tile) * plan->kblocks, T, G);
+        const bool whole = kb0 == 0 && kb1 == plan->kblocks;
+        if (n < max) {
+            out[n].tile_row = 0;
+            out[n].tile_col = tile;
+            out[n].kb_begin = kb0;
+            out[n].kb_end = kb1;
+            out[n].split = whole ? -1 : cta - first;
+        }
+        ++n;
+        it += kb1 - kb0;
+    }
+    return n;
+}
+
 gemm_status_t gemm_relu_plan_unit(const gemm_relu_plan_t *plan, int u, gemm_relu_unit_t *unit)
 {
-    if (!plan || !unit || u < 0 || u >= plan->units || plan->split_k < 1 || plan->panel < 1)
+    if (!plan || !unit || u < 0 || u >= plan->units || plan->split_k < 1 || plan->panel < 1 ||
+        plan->stream_k > 0)
         return GEMM_ERR_INVALID_ARG;
     const WorkUnit w = decode_unit(u, plan->tiles_m, plan->tiles_n, plan->split_k, plan->kblocks,
                                    plan->panel);

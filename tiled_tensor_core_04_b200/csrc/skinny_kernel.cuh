@@ -18,8 +18,16 @@
 //     NP-column buffers so the epilogue overlaps the next tile.
 //   Epilogue: lane t of warp q holds C[:, n0 + 32q + t]; for each m it writes
 //     C[m, n] -- 32 consecutive n per warp store, i.e. coalesced rows of C.
-//   Split-K: as in the main kernel, fp32 partials (no ReLU) per split, added
-//     in split order by the reduction kernel.
+//   Split-K (default when the column tiles cannot fill the SMs): K is cut in
+//     S equal ranges, each written as a fp32 partial slice, all CTAs walking
+//     K in step (DRAM pages of B are read by neighbouring CTAs together); the
+//     slices are added in split order by splitk_reduce_kernel.
+//   Stream-K (option): the T = tiles * kblocks K blocks are spread evenly
+//     over all CTAs (one contiguous range each).  A tile whose
+//     whole K range one CTA owns is written to C directly (ReLU + cast); a
+//     tile split between CTAs leaves one fp32 partial per piece in numbered
+//     slots, and streamk_reduce_kernel adds the pieces in slot order, then
+//     applies the ReLU and the cast (deterministic).
 //   Slot release in groups: the ring is released kGroup stages at a time
 //     (one tcgen05.commit per kGroup stages, one "empty" barrier per group)
 //     while each stage keeps its own "full" barrier, so the MMA issuer pays
@@ -44,6 +52,48 @@ struct SkinnyCfg {
     static constexpr int kGroups = kStages / kGroup;
     static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
     static constexpr uint32_t kTmemCols = 2 * NP < 32 ? 32 : 2 * NP;   // power of two
+};
+
+// The work of one CTA, piece by piece: whole tiles (u = blockIdx.x, +gridDim.x)
+// or, in stream-K mode, the tile segments of its iteration range.  All three
+// roles walk the same sequence.
+struct SkinnyWork {
+    int64_t it, end;   // stream-K iteration cursor
+    int u;             // tile cursor otherwise
+    __device__ __forceinline__ void start(const GemmParams &p)
+    {
+        if (p.sk_iters > 0) {
+            it = sk_begin(blockIdx.x, p.sk_iters, gridDim.x);
+            end = sk_begin(blockIdx.x + 1, p.sk_iters, gridDim.x);
+        } else {
+            u = blockIdx.x;
+        }
+    }
+    // next piece: column tile, K blocks [kb0, kb1), slot index, whole-tile flag
+    __device__ __forceinline__ bool next(const GemmParams &p, WorkUnit &w, int &slot, bool &whole)
+    {
+        if (p.sk_iters > 0) {
+            if (it >= end) return false;
+            const int tile = static_cast<int>(it / p.kblocks);
+            w.m_tile = 0;
+            w.n_tile = tile;
+            w.split = 0;
+            w.kb0 = static_cast<int>(it - static_cast<int64_t>(tile) * p.kblocks);
+            const int64_t left = end - it;
+            w.kb1 = static_cast<int>(min(static_cast<int64_t>(p.kblocks), w.kb0 + left));
+            const int first = sk_owner(static_cast<int64_t>(tile) * p.kblocks, p.sk_iters, gridDim.x);
+            slot = tile * p.sk_max_seg + (static_cast<int>(blockIdx.x) - first);
+            whole = (w.kb0 == 0 && w.kb1 == p.kblocks);
+            it += w.kb1 - w.kb0;
+            return true;
+        }
+        if (u >= p.num_units) return false;
+        w = decode_unit(u, p.tiles_m, p.tiles_n, p.splits, p.kblocks, p.panel);
+        slot = w.split;
+        whole = p.splits == 1;
+        u += gridDim.x;
+        return true;
+    }
 };
 
 template <int NP, bool B_MN, typename OutT>
@@ -105,8 +155,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             int stage = 0;
             uint32_t phase = 0;
             uint32_t issued_mask = 0, last_parity = 0;
-            for (int u = blockIdx.x; u < p.num_units && !aborted; u += gridDim.x) {
-                const WorkUnit w = decode_unit(u, p.tiles_m, p.tiles_n, p.splits, p.kblocks, p.panel);
+            SkinnyWork work;
+            work.start(p);
+            WorkUnit w;
+            int slot;
+            bool whole;
+            while (!aborted && work.next(p, w, slot, whole)) {
                 const int n0 = w.n_tile * Cfg::kTileN;
                 for (int kb = w.kb0; kb < w.kb1; ++kb) {
                     // a whole group of slots is released by one commit
@@ -160,8 +214,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             // whether the next slot's operands were seen to have landed (peeked
             // before the current slot's MMAs are issued)
             bool next_ready = mbar_test_wait(smem_addr(&full_bar[0]), 0);
-            for (int u = blockIdx.x; u < p.num_units && !aborted; u += gridDim.x, ++local) {
-                const WorkUnit w = decode_unit(u, p.tiles_m, p.tiles_n, p.splits, p.kblocks, p.panel);
+            SkinnyWork work;
+            work.start(p);
+            WorkUnit w;
+            int slot;
+            bool whole;
+            for (; !aborted && work.next(p, w, slot, whole); ++local) {
                 const int buf = local & 1;
                 const uint32_t tphase = static_cast<uint32_t>(local >> 1) & 1u;
                 if (!wait_phase_thread<false>(smem_addr(&tempty_bar[buf]), tphase ^ 1u, wc,
@@ -205,8 +263,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------ epilogue (warps 2..5)
         const int q = warp & 3;
         int local = 0;
-        for (int u = blockIdx.x; u < p.num_units && !aborted; u += gridDim.x, ++local) {
-            const WorkUnit w = decode_unit(u, p.tiles_m, p.tiles_n, p.splits, p.kblocks, p.panel);
+        SkinnyWork work;
+        work.start(p);
+        WorkUnit w;
+        int slot;
+        bool whole;
+        for (; !aborted && work.next(p, w, slot, whole); ++local) {
             const int buf = local & 1;
             const uint32_t tphase = static_cast<uint32_t>(local >> 1) & 1u;
             if (!wait_phase<false>(smem_addr(&tfull_bar[buf]), tphase, wc, kErrEpilogue)) {
@@ -214,9 +276,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after_sync();
-            const int n = w.n_tile * Cfg::kTileN + q * 32 + lane;   // column of C
+            const int n_local = q * 32 + lane;
+            const int n = w.n_tile * Cfg::kTileN + n_local;   // column of C
             const bool n_ok = n < p.N;
-            OutT *out = reinterpret_cast<OutT *>(p.C) + static_cast<int64_t>(w.split) * p.split_stride;
+            OutT *out = reinterpret_cast<OutT *>(p.C);
+            // partials: stream-K slot (M x 128, pitch 128) or split-K slice (M x N, pitch N)
+            float *part = nullptr;
+            int64_t part_pitch = 0;
+            int part_col = 0;
+            if (!whole) {
+                if (p.sk_iters > 0) {
+                    part = p.sk_ws + static_cast<int64_t>(slot) * p.M * Cfg::kTileN;
+                    part_pitch = Cfg::kTileN;
+                    part_col = n_local;
+                } else {
+                    part = p.sk_ws + static_cast<int64_t>(slot) * p.split_stride;
+                    part_pitch = p.N;
+                    part_col = n;
+                }
+            }
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                    static_cast<uint32_t>(buf * NP);
 #pragma unroll 1
@@ -228,10 +306,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int m = c + i;
-                    if (n_ok && m < p.M) {
+                    if (m < p.M) {
                         float x = __uint_as_float(v[i]);
-                        if (p.relu) x = fmaxf(x, 0.0f);
-                        out[static_cast<int64_t>(m) * p.ldc + n] = convert_out<OutT>(x);
+                        if (!whole) {
+                            if (p.sk_iters > 0 || n_ok)
+                                part[m * part_pitch + part_col] = x;   // raw partial, no ReLU
+                        } else if (n_ok) {
+                            if (p.relu) x = fmaxf(x, 0.0f);
+                            out[static_cast<int64_t>(m) * p.ldc + n] = convert_out<OutT>(x);
+                        }
                     }
                 }
             }
