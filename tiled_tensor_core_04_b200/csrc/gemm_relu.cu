@@ -521,12 +521,9 @@ uint32_t make_idesc(gemm_dtype_t in, bool b_mn, int mma_m, int mma_n, bool a_mn 
 }
 
 gemm_status_t launch_repitch(const void *src, int64_t rows, int64_t cols, void *dst,
-                             int64_t pitch, cudaStream_t stream)
+                             int64_t pitch, int sms, cudaStream_t stream)
 {
     // one warp per row at a time, at most 8 blocks of 8 warps per SM
-    int sms = 148;
-    int dev = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(ceil_div(rows, 8), 8LL * sms));
     repitch_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(
         static_cast<const uint16_t *>(src), rows, cols, static_cast<uint16_t *>(dst), pitch);
@@ -637,7 +634,9 @@ gemm_status_t run(const void *A, const void *B, void *C, int64_t M, int64_t N, i
     cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
     gemm_relu_plan_t plan;
     Layout lay;
-    // argument checks first (no device needed)
+    // Argument checks need no device: a plan for a nominal 148-SM part either
+    // fails on the arguments or succeeds; the real plan is made below with
+    // the current device's SM and cluster counts.
     gemm_status_t st = make_plan(M, N, K, in, out, trans_b, A, B, 148, 74, opts, &plan, &lay);
     if (st != GEMM_OK) return st;
     if (M == 0 || N == 0) return GEMM_OK;
@@ -664,7 +663,7 @@ gemm_status_t run(const void *A, const void *B, void *C, int64_t M, int64_t N, i
     const void *a_src = A;
     int64_t a_pitch = K;
     if (plan.pack_a) {
-        st = launch_repitch(A, M, K, wsb + lay.a_off, lay.a_pitch, stream);
+        st = launch_repitch(A, M, K, wsb + lay.a_off, lay.a_pitch, dev->sms, stream);
         if (st != GEMM_OK) return st;
         a_src = wsb + lay.a_off;
         a_pitch = lay.a_pitch;
@@ -672,7 +671,8 @@ gemm_status_t run(const void *A, const void *B, void *C, int64_t M, int64_t N, i
     const void *b_src = B;
     int64_t b_pitch = trans_b ? K : N;
     if (plan.pack_b) {
-        st = launch_repitch(B, trans_b ? N : K, trans_b ? K : N, wsb + lay.b_off, lay.b_pitch, stream);
+        st = launch_repitch(B, trans_b ? N : K, trans_b ? K : N, wsb + lay.b_off, lay.b_pitch,
+                            dev->sms, stream);
         if (st != GEMM_OK) return st;
         b_src = wsb + lay.b_off;
         b_pitch = lay.b_pitch;
