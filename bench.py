@@ -237,7 +237,8 @@ def workload_config(w: wl.Workload, args) -> dict:
             "l2": ("inputs larger than L2 (A+B = %d MB > 126 MB), no flush"
                    % ((w.M * w.K + w.N * w.K) * 2 // 2 ** 20))
             if (w.M * w.K + w.N * w.K) * 2 > L2_BYTES else "L2 flushed between steps",
-            "parallelism": f"{args.gpus} independent replica(s), one per GPU"}
+            "parallelism": f"{args.gpus} independent replica(s), one per GPU",
+            **({"options": json.loads(args.options)} if getattr(args, "options", "") else {})}
 
 
 def bench_ours(args, world, rank, local):
@@ -255,8 +256,16 @@ def bench_ours(args, world, rank, local):
     stream = torch.cuda.Stream(device=dev)
     sptr = stream.cuda_stream
     props = torch.cuda.get_device_properties(dev)
+    opts = json.loads(args.options) if args.options else None
     plan = g.gemm_relu_plan(w.M, w.N, w.K, w.in_dtype, w.out_dtype, w.trans_b, A, B,
-                            num_sms=props.multi_processor_count)
+                            num_sms=props.multi_processor_count, options=opts)
+
+    def call(a, b, c):
+        if opts is None:   # the plain C entry point
+            g.gemm_relu(a, b, c, w.M, w.N, w.K, w.in_dtype, w.out_dtype, w.trans_b, w.relu, sptr)
+        else:
+            g.gemm_relu_ex(a, b, c, w.M, w.N, w.K, w.in_dtype, w.out_dtype, w.trans_b, w.relu,
+                           sptr, options=opts)
     launches_per_step = 1 + plan["pack_a"] + plan["pack_b"] + (1 if plan["split_k"] > 1 else 0)
 
     flush = None
@@ -266,7 +275,7 @@ def bench_ours(args, world, rank, local):
     def step():
         if flush is not None:
             flush.fill_(1)
-        g.gemm_relu(A, B, C, w.M, w.N, w.K, w.in_dtype, w.out_dtype, w.trans_b, w.relu, sptr)
+        call(A, B, C)
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
@@ -291,8 +300,7 @@ def bench_ours(args, world, rank, local):
                 if flush is not None:
                     flush.fill_(1)
                 starts[i].record(stream)
-                g.gemm_relu(A, B, C, w.M, w.N, w.K, w.in_dtype, w.out_dtype, w.trans_b, w.relu,
-                            sptr)
+                call(A, B, C)
                 ends[i].record(stream)
             t_end.record(stream)
         torch.cuda.synchronize()
@@ -341,8 +349,7 @@ def bench_ours(args, world, rank, local):
             stream.wait_event(ev_in[j])
             if ev_out[j] is not None:
                 stream.wait_event(ev_out[j])         # C[j] of step i-2 has been copied out
-            g.gemm_relu(As[j], Bs[j], Cs[j], w.M, w.N, w.K, w.in_dtype, w.out_dtype, w.trans_b,
-                        w.relu, sptr)
+            call(As[j], Bs[j], Cs[j])
             ev_done[j] = torch.cuda.Event()
             ev_done[j].record(stream)
             with torch.cuda.stream(s_out):
@@ -415,6 +422,9 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0,
                     help="seconds of oracle work for the cpu_baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--options", default="",
+                    help='JSON object of gemm_relu_options_t fields, e.g. \'{"panel": 4}\'; '
+                         "the call then goes through gemm_relu_ex")
     ap.add_argument("--reference-rows", type=int, default=1,
                     help="output rows per step of the reference (CPU oracle) arm")
     args = ap.parse_args()

@@ -60,17 +60,27 @@ def plan(w: wl.Workload, **opt):
 
 
 def test_plans_for_the_workloads(lib):
+    # 256 x 512 pair tiles: 512 units = 7 waves of 74 pairs, as many as 14 waves of 256 x 256
     p = plan(wl.WORKLOADS["square8192_f16"])
-    assert (p["cta_pair"], p["tile_m"], p["tile_n"], p["split_k"]) == (1, 256, 256, 1)
-    assert (p["tile_k"], p["kblocks"], p["stages"]) == (128, 64, 3)
-    assert (p["tiles_m"], p["tiles_n"], p["units"], p["grid_ctas"]) == (32, 32, 1024, 148)
+    assert (p["cta_pair"], p["tile_m"], p["tile_n"], p["split_k"]) == (1, 256, 512, 1)
+    assert (p["tile_k"], p["kblocks"], p["stages"]) == (64, 128, 4)
+    assert (p["tiles_m"], p["tiles_n"], p["units"], p["grid_ctas"]) == (32, 16, 512, 148)
     assert p["pack_a"] == p["pack_b"] == 0 and p["workspace_bytes"] == 0
+    p = plan(wl.WORKLOADS["square8192_f16"], wide=2)
+    assert (p["tile_n"], p["tile_k"], p["kblocks"], p["stages"]) == (256, 128, 64, 3)
+    assert (p["tiles_m"], p["tiles_n"], p["units"], p["grid_ctas"]) == (32, 32, 1024, 148)
 
+    # 14 wide columns would need 7 waves (= 14 of 256 x 256), 28 narrow ones 13
     p = plan(wl.WORKLOADS["bt8192x7168x8192_bf16_f32"])
-    assert p["cta_pair"] == 1 and p["tiles_n"] == 28 and p["units"] == 896
+    assert p["cta_pair"] == 1 and p["tile_n"] == 256 and p["tiles_n"] == 28 and p["units"] == 896
+    p = plan(wl.WORKLOADS["bt8192x7168x8192_bf16_f32"], wide=1)
+    assert p["tile_n"] == 512 and p["tiles_n"] == 14 and p["units"] == 448
 
     p = plan(wl.WORKLOADS["tail5000x3001x2050_f16"])
     assert p["pack_a"] == 1 and p["pack_b"] == 1          # 4100- and 6002-byte row pitches
+    assert p["tile_n"] == 512 and p["tiles_m"] == 20 and p["tiles_n"] == 6
+    assert p["kblocks"] == 33                              # K tail 2050 % 64
+    p = plan(wl.WORKLOADS["tail5000x3001x2050_f16"], wide=2)
     assert p["kblocks"] == 17 and p["tiles_m"] == 20 and p["tiles_n"] == 12   # K tail 2050 % 128
 
     p = plan(wl.WORKLOADS["skinny64x8192x8192_f16"])
@@ -106,7 +116,14 @@ def test_options_override_the_plan(lib):
     assert plan(w, force_pack=1)["pack_a"] == 1
     assert plan(w, panel=3)["panel"] == 3
     p = plan(w, stage_k=64)
-    assert (p["tile_k"], p["kblocks"], p["stages"]) == (64, 64, 7)
+    assert (p["tile_n"], p["tile_k"], p["kblocks"], p["stages"]) == (256, 64, 64, 7)
+    assert plan(w)["tile_n"] == 512                          # 2 waves of wide tiles = 4 narrow
+    assert plan(w, wide=2)["tile_n"] == 256
+    assert plan(w, split_k=2, wide=1)["tile_n"] == 256       # no split-K on the wide kernel
+    assert plan(w, cta_pair=g.GEMM_CTA_SINGLE, wide=1)["tile_n"] == 256
+    assert plan(w, stage_k=128)["tile_n"] == 256
+    with pytest.raises(g.GemmError):
+        plan(w, wide=3)
     assert plan(w, cta_pair=g.GEMM_CTA_SINGLE, stage_k=128)["tile_k"] == 64   # 1-CTA: 64 only
     with pytest.raises(g.GemmError):
         plan(w, stage_k=96)

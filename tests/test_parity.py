@@ -104,6 +104,9 @@ VARIANTS = {
     "swap_streamk": {"swap_ab": 1, "stream_k": 1},
     "swap_streamk_few": {"swap_ab": 1, "stream_k": 1, "max_ctas": 7},
     "no_swap": {"swap_ab": 2},
+    "wide": {"cta_pair": g.GEMM_CTA_PAIR, "wide": 1},
+    "wide_few": {"cta_pair": g.GEMM_CTA_PAIR, "wide": 1, "max_ctas": 4, "panel": 3},
+    "no_wide": {"wide": 2},
 }
 
 
@@ -184,8 +187,20 @@ def test_full_size_workloads_sampled(name):
     sampled_check(w, C, A, B)
 
 
+@pytest.mark.parametrize("name,opt", [("square8192_f16", "no_wide"),
+                                      ("bt8192x7168x8192_bf16_f32", "wide"),
+                                      ("tail5000x3001x2050_f16", "no_wide")])
+def test_full_size_workloads_other_tile(name, opt):
+    # the tile shape the planner did not pick for this workload
+    w = wl.WORKLOADS[name]
+    A, B = wl.workload_inputs(w)
+    C = run(A, B, w.out_dtype, w.trans_b, True, VARIANTS[opt])
+    assert torch.isfinite(C.float()).all() and (C.float() >= 0).all()
+    sampled_check(w, C, A, B)
+
+
 # ---------------------------------------------------------------- closed forms
-@pytest.mark.parametrize("variant", ["auto", "single", "split3", "pair_k64"])
+@pytest.mark.parametrize("variant", ["auto", "single", "split3", "pair_k64", "wide", "wide_few"])
 @pytest.mark.parametrize("trans_b", [False, True])
 @pytest.mark.parametrize("M,N,K", [(300, 520, 2050), (256, 512, 8192), (70, 33, 9)])
 def test_ones_give_exactly_K(M, N, K, trans_b, variant):
@@ -214,7 +229,8 @@ def test_all_negative_product_is_zero(trans_b):
     assert (C.float() == 0).all()
 
 
-@pytest.mark.parametrize("variant", ["auto", "single", "split3", "packed", "pair_k64"])
+@pytest.mark.parametrize("variant", ["auto", "single", "split3", "packed", "pair_k64", "wide",
+                                     "no_wide"])
 @pytest.mark.parametrize("trans_b", [False, True])
 @pytest.mark.parametrize("in_dtype", [F16, BF16])
 @pytest.mark.parametrize("M,N,K", [(300, 520, 1000), (129, 264, 72), (5000 // 8, 3001, 2050)])

@@ -59,6 +59,7 @@ class GemmOptions(ctypes.Structure):
         ("wait_sleep_ns", ctypes.c_uint32),
         ("swap_ab", ctypes.c_int),
         ("stream_k", ctypes.c_int),
+        ("wide", ctypes.c_int),
     ]
 
 

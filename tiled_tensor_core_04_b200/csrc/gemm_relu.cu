@@ -17,6 +17,7 @@
 #include "aux_kernels.cuh"
 #include "gemm_kernel.cuh"
 #include "skinny_kernel.cuh"
+#include "wide_kernel.cuh"
 
 namespace {
 
@@ -75,6 +76,22 @@ int variant_index(bool pair, int kk, bool b_mn, gemm_dtype_t out)
 {
     const int shape = pair ? (kk == 2 ? 2 : 1) : 0;
     return shape * 6 + (b_mn ? 3 : 0) + static_cast<int>(out);
+}
+
+// Wide CTA-pair kernels (256 x 512 tiles): B MN- or K-major, three output types.
+template <bool BMN>
+GemmKernelFn pick_wide_out(gemm_dtype_t out)
+{
+    switch (out) {
+    case GEMM_F16: return gemm_relu_wide_kernel<BMN, __half>;
+    case GEMM_BF16: return gemm_relu_wide_kernel<BMN, __nv_bfloat16>;
+    default: return gemm_relu_wide_kernel<BMN, float>;
+    }
+}
+
+GemmKernelFn pick_wide(bool b_mn, gemm_dtype_t out)
+{
+    return b_mn ? pick_wide_out<true>(out) : pick_wide_out<false>(out);
 }
 
 // Skinny-M (swap-AB) kernels: NP in {16, 32, 64, 128}, B MN- or K-major.
@@ -139,6 +156,7 @@ struct DeviceInfo {
     int max_pair_clusters = 0;
     bool attr_set[18] = {};
     bool skinny_attr_set[24] = {};
+    bool wide_attr_set[6] = {};
 };
 
 std::mutex g_dev_mutex;
@@ -165,6 +183,18 @@ gemm_status_t ensure_skinny_attr(DeviceInfo &d, int np, bool b_mn, gemm_dtype_t 
                                          skinny_smem(np));
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(skinny)");
     d.skinny_attr_set[v] = true;
+    return GEMM_OK;
+}
+
+gemm_status_t ensure_wide_attr(DeviceInfo &d, bool b_mn, gemm_dtype_t out)
+{
+    const int v = (b_mn ? 3 : 0) + static_cast<int>(out);
+    if (d.wide_attr_set[v]) return GEMM_OK;
+    cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void *>(pick_wide(b_mn, out)),
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         WideCfg::kSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(wide)");
+    d.wide_attr_set[v] = true;
     return GEMM_OK;
 }
 
@@ -245,7 +275,7 @@ gemm_status_t make_plan(int64_t M, int64_t N, int64_t K, gemm_dtype_t in, gemm_d
     if (o.cta_pair < 0 || o.cta_pair > 2 || o.split_k < 0 || o.panel < 0 || o.max_ctas < 0 ||
         (o.stage_k != 0 && o.stage_k != 64 && o.stage_k != 128) || o.l2_hint_a < 0 ||
         o.l2_hint_a > 2 || o.l2_hint_b < 0 || o.l2_hint_b > 2 || o.c_streaming < 0 || o.c_streaming > 1 || o.swap_ab < 0 || o.swap_ab > 2 ||
-        o.stream_k < 0 || o.stream_k > 1)
+        o.stream_k < 0 || o.stream_k > 1 || o.wide < 0 || o.wide > 2)
         return GEMM_ERR_INVALID_ARG;
 
     gemm_relu_plan_t p = {};
@@ -326,26 +356,42 @@ gemm_status_t make_plan(int64_t M, int64_t N, int64_t K, gemm_dtype_t in, gemm_d
 
     p.cta_pair = pair ? 1 : 0;
     p.tile_m = pair ? 2 * kBM : kBM;
-    // the pair kernel takes 128 of K per pipeline stage unless asked for 64
-    const int kk = (pair && o.stage_k != 64) ? 2 : 1;
+    const int64_t tiles_m = ceil_div(M, p.tile_m);
+    int64_t clusters = max_pair_clusters > 0 ? max_pair_clusters : num_sms / 2;
+    if (o.max_ctas > 0) clusters = std::min<int64_t>(clusters, std::max(1, o.max_ctas / 2));
+    clusters = std::max<int64_t>(1, clusters);
+    // 256 x 512 pair tiles: half the units, each twice the work; taken when
+    // that costs no more waves of units than 256 x 256 tiles
+    bool wide = false;
+    if (pair && split == 1 && o.wide != 2) {
+        if (o.wide == 1)
+            wide = true;
+        else if (o.stage_k == 0) {
+            const int64_t waves_sq = ceil_div(tiles_m * tiles_n, clusters);
+            const int64_t waves_wide = ceil_div(tiles_m * ceil_div(N, 2 * kBN), clusters);
+            wide = 2 * waves_wide <= waves_sq;
+        }
+    }
+    // the 256 x 256 pair kernel takes 128 of K per pipeline stage unless asked
+    // for 64; the wide kernel takes 64
+    const int kk = (pair && !wide && o.stage_k != 64) ? 2 : 1;
     p.tile_k = kBK * kk;
     p.kblocks = static_cast<int>(ceil_div(K, p.tile_k));
-    const int64_t tiles_m = ceil_div(M, p.tile_m);
-    const int64_t units = tiles_m * tiles_n * split;
+    if (wide) p.tile_n = 2 * kBN;
+    const int64_t tiles_n_used = wide ? ceil_div(N, 2 * kBN) : tiles_n;
+    const int64_t units = tiles_m * tiles_n_used * split;
     if (units > INT32_MAX) return GEMM_ERR_INVALID_ARG;
     p.tiles_m = static_cast<int>(tiles_m);
-    p.tiles_n = static_cast<int>(tiles_n);
+    p.tiles_n = static_cast<int>(tiles_n_used);
     p.split_k = static_cast<int>(split);
     p.panel = o.panel > 0 ? o.panel : kDefaultPanel;
     if (p.tiles_m > 0) p.panel = std::min(p.panel, p.tiles_m);
     p.units = static_cast<int>(units);
-    p.stages = stage_count(pair, kk);
+    p.stages = wide ? WideCfg::kStages : stage_count(pair, kk);
 
     int64_t grid;
     if (pair) {
-        int64_t clusters = max_pair_clusters > 0 ? max_pair_clusters : num_sms / 2;
-        if (o.max_ctas > 0) clusters = std::min<int64_t>(clusters, std::max(1, o.max_ctas / 2));
-        grid = 2 * std::min<int64_t>(units, std::max<int64_t>(1, clusters));
+        grid = 2 * std::min<int64_t>(units, clusters);
     } else {
         int64_t ctas = num_sms;
         if (o.max_ctas > 0) ctas = std::min<int64_t>(ctas, o.max_ctas);
@@ -719,16 +765,17 @@ gemm_status_t run(const void *A, const void *B, void *C, int64_t M, int64_t N, i
     p.c_stream = (!split && opts) ? opts->c_streaming : 0;
     p.sleep_ns = (opts && opts->wait_sleep_ns) ? opts->wait_sleep_ns : 0;
 
+    const bool wide = plan.tile_n == WideCfg::kTileN;
     {
         std::lock_guard<std::mutex> lock(g_dev_mutex);
-        st = ensure_kernel_attr(*dev, pair, kk, b_mn, kout);
+        st = wide ? ensure_wide_attr(*dev, b_mn, kout) : ensure_kernel_attr(*dev, pair, kk, b_mn, kout);
     }
     if (st != GEMM_OK) return st;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(plan.grid_ctas), 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem_bytes(pair, kk);
+    cfg.blockDim = dim3(wide ? kWideThreads : kThreads, 1, 1);
+    cfg.dynamicSmemBytes = wide ? WideCfg::kSmemBytes : smem_bytes(pair, kk);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -737,7 +784,8 @@ gemm_status_t run(const void *A, const void *B, void *C, int64_t M, int64_t N, i
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pair ? 1 : 0;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, pick_kernel(pair, kk, b_mn, kout), tmA, tmB, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, wide ? pick_wide(b_mn, kout) : pick_kernel(pair, kk, b_mn, kout),
+                                       tmA, tmB, p);
     if (e != cudaSuccess) return cuda_fail(e, "gemm kernel launch");
 
     if (split) {

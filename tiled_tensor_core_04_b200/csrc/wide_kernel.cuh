@@ -1,0 +1,293 @@
+// wide_kernel.cuh -- the 256 x 512 CTA-pair variant of the fused GEMM + ReLU
+// tile loop (the "Tiled GEMM with a fused ReLU epilogue" example of the
+// TileLang notes, T.gemm into a fragment accumulator, T.max(C, 0) on the way
+// out, computed here with tcgen05 tensor cores).
+//
+// Same roles, barriers and bounded waits as gemm_kernel.cuh; what differs:
+//  * One unit is a 256 x 512 tile of C.  Each CTA of the pair holds 128 rows
+//    of A and 256 of the tile's columns of B (128 of each 256-column half);
+//    every K step issues two cta_group::2 MMAs of M = 256, N = 256, one per
+//    half.  Per flop, the pair reads 25 % fewer operand bytes from L2 than a
+//    256 x 256 tile, and one wave of tiles touches fewer DRAM bytes.
+//  * The fp32 accumulator fills all 512 TMEM columns, so there is a single
+//    accumulator, released in two 256-column halves: the epilogue drains
+//    half 0, frees it, then half 1.  At the start of a unit the MMA warp
+//    issues half 0 of the first `kStages` K blocks (all in shared memory
+//    already) before it needs half 1 back, so draining half 1 overlaps MMA
+//    work; only the drain of half 0 is exposed.
+//  * Eight epilogue warps (two per TMEM lane quarter, 128 columns of a half
+//    each) halve the drain time.
+//  * One split only (no split-K); K blocks of 64 per stage, 48 KB per stage
+//    per CTA, 4 stages.
+#pragma once
+
+#include "gemm_kernel.cuh"
+
+namespace gr {
+
+constexpr int kWideThreads = 320;  // producer, MMA, 8 epilogue warps
+constexpr int kWideEpiWarps = 8;
+
+struct WideCfg {
+    static constexpr int kTileM = 2 * kBM;                  // 256 rows per CTA pair
+    static constexpr int kTileN = 2 * kBN;                  // 512 columns: two MMA halves
+    static constexpr int kABytes = kBM * kBK * 2;           // 16 KB: 128 rows x 64 K
+    static constexpr int kBHalf = (kBN / 2) * kBK * 2;      // 16 KB: 128 columns x 64 K
+    static constexpr int kStageBytes = kABytes + 2 * kBHalf;  // 48 KB
+    static constexpr int kStagesFit = (232448 - 2048) / kStageBytes;
+    static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
+    // the loads of both CTAs complete on the leader's barrier
+    static constexpr uint32_t kTxBytes = 2 * kStageBytes;
+    static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
+};
+
+template <bool B_MN, typename OutT>
+__global__ void __launch_bounds__(kWideThreads, 1)
+    gemm_relu_wide_kernel(const __grid_constant__ CUtensorMap tmA,
+                          const __grid_constant__ CUtensorMap tmB, const GemmParams p)
+{
+    using Cfg = WideCfg;
+    constexpr int kStages = Cfg::kStages;
+
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t full_bar[kStages];
+    __shared__ __align__(8) uint64_t empty_bar[kStages];
+    __shared__ __align__(8) uint64_t tfull_bar[2];   // per accumulator half
+    __shared__ __align__(8) uint64_t tempty_bar[2];  // per accumulator half
+    __shared__ __align__(8) uint64_t drain_bar;
+    __shared__ uint32_t tmem_slot;
+    __shared__ int abort_flag;
+
+    const int warp = static_cast<int>(threadIdx.x >> 5);
+    const int lane = static_cast<int>(threadIdx.x & 31);
+    const uint32_t rank = cluster_cta_rank();
+    const uint32_t tiles_base = (smem_addr(smem_raw) + 1023u) & ~1023u;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(smem_addr(&full_bar[s]), 1);
+            mbar_init(smem_addr(&empty_bar[s]), 1);
+        }
+        for (int h = 0; h < 2; ++h) {
+            mbar_init(smem_addr(&tfull_bar[h]), 1);
+            mbar_init(smem_addr(&tempty_bar[h]), 2 * kWideEpiWarps);  // both CTAs' epilogue warps
+        }
+        mbar_init(smem_addr(&drain_bar), 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensor_map(&tmA);
+        prefetch_tensor_map(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc<2>(smem_addr(&tmem_slot), kTmemCols);
+        tmem_relinquish<2>();
+    }
+    tc_fence_before_sync();
+    cluster_sync_all();
+    tc_fence_after_sync();
+    const uint32_t tmem_base = tmem_slot;
+
+    const WaitCtx wc{&abort_flag, p.timeout_ns, p.sleep_ns};
+    const int cluster_id = static_cast<int>(blockIdx.x >> 1);
+    const int num_clusters = static_cast<int>(gridDim.x >> 1);
+    bool aborted = false;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer (one lane)
+        if (lane == 0) {
+            const uint64_t pol_a = make_l2_policy(p.l2_a);
+            const uint64_t pol_b = make_l2_policy(p.l2_b);
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued_mask = 0;
+            uint32_t last_parity = 0;
+            int local = 0;
+            for (int u = cluster_id; u < p.num_units && !aborted; u += num_clusters, ++local) {
+                const WorkUnit w = decode_unit(u, p.tiles_m, p.tiles_n, 1, p.kblocks, p.panel);
+                const int m_row = w.m_tile * Cfg::kTileM + static_cast<int>(rank) * kBM;
+                const int n_col = w.n_tile * Cfg::kTileN + static_cast<int>(rank) * (kBN / 2);
+                for (int i = 0; i < w.kb1 - w.kb0; ++i) {
+                    const int kb = k_block_at(w, i, local);
+                    if (!wait_phase_thread<false>(smem_addr(&empty_bar[stage]), phase ^ 1u, wc,
+                                                  kErrProducer)) {
+                        aborted = true;
+                        break;
+                    }
+                    const uint32_t fb = smem_addr(&full_bar[stage]);
+                    const uint32_t fb_leader = map_shared_to_rank(fb, 0);
+                    const uint32_t a_dst = tiles_base + static_cast<uint32_t>(stage * Cfg::kStageBytes);
+                    const uint32_t b_dst = a_dst + Cfg::kABytes;
+                    const int kx = kb * kBK;
+                    if (rank == 0) mbar_arrive_expect_tx(fb, Cfg::kTxBytes);
+                    tma_load_2d_pair_hint(a_dst, &tmA, fb_leader, kx, m_row, pol_a);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int n = n_col + h * kBN;
+                        const uint32_t dst = b_dst + static_cast<uint32_t>(h * Cfg::kBHalf);
+                        if constexpr (B_MN) {
+                            tma_load_2d_pair_hint(dst, &tmB, fb_leader, n, kx, pol_b);
+                            tma_load_2d_pair_hint(dst + 8192, &tmB, fb_leader, n + 64, kx, pol_b);
+                        } else {
+                            tma_load_2d_pair_hint(dst, &tmB, fb_leader, kx, n, pol_b);
+                        }
+                    }
+                    issued_mask |= 1u << stage;
+                    last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (aborted && rank == 0) {
+                for (int s = 0; s < kStages; ++s)
+                    if (issued_mask & (1u << s))
+                        if (!wait_phase_one(smem_addr(&full_bar[s]), (last_parity >> s) & 1u, 20000000ull))
+                            atomicOr(&g_gemm_device_error, kErrDrain);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer (one lane of the leader)
+        if (rank == 0 && lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int local = 0;
+            bool issued_any = false;
+            const uint64_t a_desc0 = smem_desc_sw128(tiles_base, 16, 1024);
+            const uint64_t b_desc0 = B_MN ? smem_desc_sw128(tiles_base + Cfg::kABytes, 8192, 1024)
+                                          : smem_desc_sw128(tiles_base + Cfg::kABytes, 16, 1024);
+            constexpr uint64_t kAStep = 32 >> 4;                         // 16 K of a K-major row
+            constexpr uint64_t kBStep = B_MN ? (2048 >> 4) : (32 >> 4);  // 16 K rows / elements
+            constexpr uint64_t kStageStep = Cfg::kStageBytes >> 4;
+            constexpr uint64_t kHalfStep = Cfg::kBHalf >> 4;
+            const uint32_t idesc = p.idesc;
+            // four K = 16 MMAs of one stage into accumulator half h
+            auto issue_half = [&](int s, int h, bool first) {
+                const uint64_t so = static_cast<uint64_t>(s) * kStageStep;
+                const uint32_t d = tmem_base + static_cast<uint32_t>(h * kBN);
+#pragma unroll
+                for (int k = 0; k < kBK / 16; ++k)
+                    umma_f16<2>(d, a_desc0 + so + static_cast<uint64_t>(k) * kAStep,
+                                b_desc0 + so + static_cast<uint64_t>(h) * kHalfStep +
+                                    static_cast<uint64_t>(k) * kBStep,
+                                idesc, (first && k == 0) ? 0u : 1u);
+            };
+            auto advance = [&](int &s, uint32_t &ph) {
+                if (++s == kStages) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            };
+            for (int u = cluster_id; u < p.num_units && !aborted; u += num_clusters, ++local) {
+                const WorkUnit w = decode_unit(u, p.tiles_m, p.tiles_n, 1, p.kblocks, p.panel);
+                const uint32_t tphase = static_cast<uint32_t>(local) & 1u;
+                const int nkb = w.kb1 - w.kb0;
+                const int pre = nkb < kStages ? nkb : kStages;
+                // half 0 of the first `pre` K blocks, once the epilogue freed half 0
+                if (!wait_phase_thread<true>(smem_addr(&tempty_bar[0]), tphase ^ 1u, wc, kErrMmaAccum)) {
+                    aborted = true;
+                    break;
+                }
+                tc_fence_after_sync();
+                int s = stage;
+                uint32_t ph = phase;
+                for (int i = 0; i < pre; ++i) {
+                    if (!wait_phase_thread<false>(smem_addr(&full_bar[s]), ph, wc, kErrMmaOperands)) {
+                        aborted = true;
+                        break;
+                    }
+                    issue_half(s, 0, i == 0);
+                    issued_any = true;
+                    advance(s, ph);
+                }
+                if (aborted) break;
+                if (pre == nkb) umma_commit_pair(smem_addr(&tfull_bar[0]), 0x3);
+                // half 1 of the same K blocks, releasing each stage after it
+                if (!wait_phase_thread<true>(smem_addr(&tempty_bar[1]), tphase ^ 1u, wc, kErrMmaAccum)) {
+                    aborted = true;
+                    break;
+                }
+                tc_fence_after_sync();
+                s = stage;
+                ph = phase;
+                for (int i = 0; i < pre; ++i) {
+                    issue_half(s, 1, i == 0);
+                    umma_commit_pair(smem_addr(&empty_bar[s]), 0x3);
+                    advance(s, ph);
+                }
+                if (pre == nkb) umma_commit_pair(smem_addr(&tfull_bar[1]), 0x3);
+                stage = s;
+                phase = ph;
+                // the rest of K: both halves per stage
+                for (int i = pre; i < nkb; ++i) {
+                    if (!wait_phase_thread<false>(smem_addr(&full_bar[stage]), phase, wc,
+                                                  kErrMmaOperands)) {
+                        aborted = true;
+                        break;
+                    }
+                    issue_half(stage, 0, false);
+                    if (i == nkb - 1) umma_commit_pair(smem_addr(&tfull_bar[0]), 0x3);
+                    issue_half(stage, 1, false);
+                    umma_commit_pair(smem_addr(&empty_bar[stage]), 0x3);
+                    if (i == nkb - 1) umma_commit_pair(smem_addr(&tfull_bar[1]), 0x3);
+                    advance(stage, phase);
+                }
+            }
+            if (aborted && issued_any) {
+                umma_commit_pair(smem_addr(&drain_bar), 0x1);
+                if (!wait_phase_one(smem_addr(&drain_bar), 0, 20000000ull))
+                    atomicOr(&g_gemm_device_error, kErrDrain);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------ epilogue (warps 2..9)
+        const int q = warp & 3;          // TMEM lane quarter this warp may access
+        const int g = (warp - 2) >> 2;   // which 128 columns of each half
+        int local = 0;
+        for (int u = cluster_id; u < p.num_units && !aborted; u += num_clusters, ++local) {
+            const WorkUnit w = decode_unit(u, p.tiles_m, p.tiles_n, 1, p.kblocks, p.panel);
+            const uint32_t tphase = static_cast<uint32_t>(local) & 1u;
+            const int row = w.m_tile * Cfg::kTileM + static_cast<int>(rank) * kBM + q * 32 + lane;
+            const bool row_ok = row < p.M;
+            OutT *rowp = reinterpret_cast<OutT *>(p.C) + static_cast<int64_t>(row) * p.ldc;
+            for (int h = 0; h < 2; ++h) {
+                if (!wait_phase<false>(smem_addr(&tfull_bar[h]), tphase, wc, kErrEpilogue)) {
+                    aborted = true;
+                    break;
+                }
+                tc_fence_after_sync();
+                const int col0 = w.n_tile * Cfg::kTileN + h * kBN + g * (kBN / 2);
+                const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                       static_cast<uint32_t>(h * kBN + g * (kBN / 2));
+#pragma unroll 1
+                for (int c = 0; c < kBN / 2; c += 32) {
+                    if (col0 + c >= p.N) break;  // warp-uniform
+                    uint32_t v[32];
+                    tmem_load_32cols(taddr + static_cast<uint32_t>(c), v);
+                    tmem_load_wait();
+                    const int valid = min(32, p.N - (col0 + c));
+                    if (row_ok)
+                        store_row32<OutT>(rowp + col0 + c, v, valid, p.vec_ok != 0, p.relu,
+                                          p.c_stream != 0);
+                }
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(map_shared_to_rank(smem_addr(&tempty_bar[h]), 0));
+            }
+        }
+    }
+
+    __syncwarp();
+    tc_fence_before_sync();
+    cluster_sync_all();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc<2>(tmem_base, kTmemCols);
+    }
+}
+
+}  // namespace gr
