@@ -106,6 +106,8 @@ VARIANTS = {
     "no_swap": {"swap_ab": 2},
     "wide": {"cta_pair": g.GEMM_CTA_PAIR, "wide": 1},
     "wide_few": {"cta_pair": g.GEMM_CTA_PAIR, "wide": 1, "max_ctas": 4, "panel": 3},
+    # evict-first stores: the wide kernel's direct (non-TMA) epilogue
+    "wide_direct": {"cta_pair": g.GEMM_CTA_PAIR, "wide": 1, "c_streaming": 1},
     "no_wide": {"wide": 2},
 }
 
@@ -261,9 +263,11 @@ def test_M_or_N_zero_is_a_no_op():
     assert (C.float() == 7).all()
 
 
+@pytest.mark.parametrize("variant", ["auto", "wide"])
 @pytest.mark.parametrize("c_offset,a_offset", [(1, 0), (0, 1), (3, 5)])
-def test_misaligned_pointers(c_offset, a_offset):
-    full_case(260, 264, 136, F16, F16, False, c_offset=c_offset, a_offset=a_offset, seed=9)
+def test_misaligned_pointers(c_offset, a_offset, variant):
+    full_case(260, 264, 136, F16, F16, False, options=VARIANTS[variant], c_offset=c_offset,
+              a_offset=a_offset, seed=9)
 
 
 def test_runs_are_deterministic():

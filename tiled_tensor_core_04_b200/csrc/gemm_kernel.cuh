@@ -78,6 +78,7 @@ struct GemmParams {
     int l2_a, l2_b;        // L2 eviction priority of the A / B loads (0 normal, 1 first, 2 last)
     int c_stream;          // 1: store C with evict-first (streaming) stores
     uint32_t sleep_ns;     // suspend-time hint for the epilogue's accumulator waits
+    int c_tma;             // wide kernel: 1 = write C through shared memory + TMA stores
     // stream-K (skinny kernel): sk_iters > 0 spreads tiles_n * kblocks K blocks
     // evenly over the CTAs; tiles split between CTAs leave fp32 partials in
     // sk_ws, slot (tile * sk_max_seg + segment), each M x 128, row pitch 128

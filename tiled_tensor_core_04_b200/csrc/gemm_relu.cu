@@ -78,9 +78,13 @@ int variant_index(bool pair, int kk, bool b_mn, gemm_dtype_t out)
     return shape * 6 + (b_mn ? 3 : 0) + static_cast<int>(out);
 }
 
-// Wide CTA-pair kernels (256 x 512 tiles): B MN- or K-major, three output types.
+// Wide CTA-pair kernels (256 x 512 tiles): B MN- or K-major, three output
+// types; the third tensor map describes C for the TMA-store epilogue.
+using WideKernelFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
+                              const GemmParams);
+
 template <bool BMN>
-GemmKernelFn pick_wide_out(gemm_dtype_t out)
+WideKernelFn pick_wide_out(gemm_dtype_t out)
 {
     switch (out) {
     case GEMM_F16: return gemm_relu_wide_kernel<BMN, __half>;
@@ -89,7 +93,7 @@ GemmKernelFn pick_wide_out(gemm_dtype_t out)
     }
 }
 
-GemmKernelFn pick_wide(bool b_mn, gemm_dtype_t out)
+WideKernelFn pick_wide(bool b_mn, gemm_dtype_t out)
 {
     return b_mn ? pick_wide_out<true>(out) : pick_wide_out<false>(out);
 }
@@ -496,11 +500,12 @@ EncodeTiledFn encode_fn()
 struct MapKey {
     const void *base;
     int64_t inner, outer, pitch;
-    int dt, box_inner, box_outer;
+    int dt, box_inner, box_outer, swizzle;
     bool operator==(const MapKey &o) const
     {
         return base == o.base && inner == o.inner && outer == o.outer && pitch == o.pitch &&
-               dt == o.dt && box_inner == o.box_inner && box_outer == o.box_outer;
+               dt == o.dt && box_inner == o.box_inner && box_outer == o.box_outer &&
+               swizzle == o.swizzle;
     }
 };
 constexpr int kMapCache = 16;
@@ -509,21 +514,25 @@ thread_local CUtensorMap t_maps[kMapCache];
 thread_local int t_map_used = 0, t_map_next = 0;
 
 gemm_status_t encode_2d_uncached(CUtensorMap *map, const void *base, gemm_dtype_t dt, int64_t inner,
-                                 int64_t outer, int64_t pitch_elems, int box_inner, int box_outer);
+                                 int64_t outer, int64_t pitch_elems, int box_inner, int box_outer,
+                                 int swizzle);
 
-// 2-D map over a row-major 16-bit matrix: inner extent `inner` (contiguous),
-// `outer` rows `pitch_elems` apart, box {box_inner, box_outer}, 128-byte swizzle,
-// out-of-range elements read as zero.
+// 2-D map over a row-major matrix of `dt`: inner extent `inner` (contiguous),
+// `outer` rows `pitch_elems` apart, box {box_inner, box_outer}, 128- or
+// 64-byte swizzle; loads read out-of-range elements as zero, stores skip them.
 gemm_status_t encode_2d(CUtensorMap *map, const void *base, gemm_dtype_t dt, int64_t inner,
-                        int64_t outer, int64_t pitch_elems, int box_inner, int box_outer)
+                        int64_t outer, int64_t pitch_elems, int box_inner, int box_outer,
+                        int swizzle = 128)
 {
-    const MapKey key{base, inner, outer, pitch_elems, static_cast<int>(dt), box_inner, box_outer};
+    const MapKey key{base, inner, outer, pitch_elems, static_cast<int>(dt), box_inner, box_outer,
+                     swizzle};
     for (int i = 0; i < t_map_used; ++i)
         if (t_map_keys[i] == key) {
             *map = t_maps[i];
             return GEMM_OK;
         }
-    gemm_status_t st = encode_2d_uncached(map, base, dt, inner, outer, pitch_elems, box_inner, box_outer);
+    gemm_status_t st = encode_2d_uncached(map, base, dt, inner, outer, pitch_elems, box_inner,
+                                          box_outer, swizzle);
     if (st != GEMM_OK) return st;
     const int slot = t_map_next;
     t_map_keys[slot] = key;
@@ -534,7 +543,8 @@ gemm_status_t encode_2d(CUtensorMap *map, const void *base, gemm_dtype_t dt, int
 }
 
 gemm_status_t encode_2d_uncached(CUtensorMap *map, const void *base, gemm_dtype_t dt, int64_t inner,
-                                 int64_t outer, int64_t pitch_elems, int box_inner, int box_outer)
+                                 int64_t outer, int64_t pitch_elems, int box_inner, int box_outer,
+                                 int swizzle)
 {
     EncodeTiledFn fn = encode_fn();
     if (!fn) {
@@ -542,12 +552,16 @@ gemm_status_t encode_2d_uncached(CUtensorMap *map, const void *base, gemm_dtype_
         return GEMM_ERR_CUDA;
     }
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(pitch_elems * 2)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(pitch_elems) *
+                             static_cast<cuuint64_t>(dt == GEMM_F32 ? 4 : 2)};
     cuuint32_t box[2] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_outer)};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(map, dt == GEMM_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                    2, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    const CUtensorMapDataType type = dt == GEMM_F32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                     : dt == GEMM_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                       : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    CUresult r = fn(map, type, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
         t_last_cuda_error = "cuTensorMapEncodeTiled failed with CUresult " + std::to_string(static_cast<int>(r));
@@ -766,6 +780,16 @@ gemm_status_t run(const void *A, const void *B, void *C, int64_t M, int64_t N, i
     p.sleep_ns = (opts && opts->wait_sleep_ns) ? opts->wait_sleep_ns : 0;
 
     const bool wide = plan.tile_n == WideCfg::kTileN;
+    // the wide kernel writes C with TMA stores of 32 x 32 boxes when C's base
+    // and row pitch are 16-byte aligned (what a tensor map needs) and no
+    // evict-first stores were asked for
+    CUtensorMap tmC = tmA;
+    p.c_tma = 0;
+    if (wide && p.vec_ok && !split && !p.c_stream) {
+        st = encode_2d(&tmC, C, out, N, M, N, 32, 32, out == GEMM_F32 ? 128 : 64);
+        if (st != GEMM_OK) return st;
+        p.c_tma = 1;
+    }
     {
         std::lock_guard<std::mutex> lock(g_dev_mutex);
         st = wide ? ensure_wide_attr(*dev, b_mn, kout) : ensure_kernel_attr(*dev, pair, kk, b_mn, kout);
@@ -784,8 +808,8 @@ gemm_status_t run(const void *A, const void *B, void *C, int64_t M, int64_t N, i
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pair ? 1 : 0;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, wide ? pick_wide(b_mn, kout) : pick_kernel(pair, kk, b_mn, kout),
-                                       tmA, tmB, p);
+    cudaError_t e = wide ? cudaLaunchKernelEx(&cfg, pick_wide(b_mn, kout), tmA, tmB, tmC, p)
+                         : cudaLaunchKernelEx(&cfg, pick_kernel(pair, kk, b_mn, kout), tmA, tmB, p);
     if (e != cudaSuccess) return cuda_fail(e, "gemm kernel launch");
 
     if (split) {

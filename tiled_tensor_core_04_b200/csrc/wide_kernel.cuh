@@ -19,6 +19,11 @@
 //    each) halve the drain time.
 //  * One split only (no split-K); K blocks of 64 per stage, 48 KB per stage
 //    per CTA, 4 stages.
+//  * Output through shared memory (when C's rows are 16-byte aligned): each
+//    epilogue warp converts its 32 rows x 32 columns, writes them into a
+//    swizzled 32 x 32 box of its own 4 KB of shared memory and one lane sends
+//    the box to C with a TMA store, so C is written in whole lines instead of
+//    one 64-byte piece per row and lane; 16-bit outputs double-buffer the box.
 #pragma once
 
 #include "gemm_kernel.cuh"
@@ -38,13 +43,51 @@ struct WideCfg {
     static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
     // the loads of both CTAs complete on the leader's barrier
     static constexpr uint32_t kTxBytes = 2 * kStageBytes;
-    static constexpr int kSmemBytes = kStages * kStageBytes + 1024;
+    static constexpr int kOutWarpBytes = 4096;  // one 32 x 32 fp32 box or two 16-bit boxes
+    static constexpr int kOutBytes = kWideEpiWarps * kOutWarpBytes;
+    static constexpr int kSmemBytes = kStages * kStageBytes + kOutBytes + 1024;
 };
+
+// One row's 32 outputs (ReLU, rounding) into a 32 x 32 staging box laid out
+// for the TMA store: 64-byte rows with the 64-byte swizzle (16-bit outputs)
+// or 128-byte rows with the 128-byte swizzle (fp32), i.e. 16-byte chunk i of
+// row r sits at chunk i ^ ((r >> 1) & 3), resp. i ^ (r & 7).  A warp storing
+// one chunk index of 32 rows then touches every bank once per 8 lanes.
+template <typename OutT>
+__device__ __forceinline__ void stage_row32(uint32_t box, int r, const uint32_t (&v)[32], int relu)
+{
+    float f[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const float x = __uint_as_float(v[i]);
+        f[i] = relu ? fmaxf(x, 0.0f) : x;
+    }
+    if constexpr (std::is_same_v<OutT, float>) {
+        const uint32_t row = box + static_cast<uint32_t>(r) * 128u;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t chunk = static_cast<uint32_t>(i ^ (r & 7));
+            st_shared_v4(row + chunk * 16u, __float_as_uint(f[4 * i]), __float_as_uint(f[4 * i + 1]),
+                         __float_as_uint(f[4 * i + 2]), __float_as_uint(f[4 * i + 3]));
+        }
+    } else {
+        const uint32_t row = box + static_cast<uint32_t>(r) * 64u;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t chunk = static_cast<uint32_t>(i ^ ((r >> 1) & 3));
+            st_shared_v4(row + chunk * 16u, pack_pair<OutT>(f[8 * i], f[8 * i + 1]),
+                         pack_pair<OutT>(f[8 * i + 2], f[8 * i + 3]),
+                         pack_pair<OutT>(f[8 * i + 4], f[8 * i + 5]),
+                         pack_pair<OutT>(f[8 * i + 6], f[8 * i + 7]));
+        }
+    }
+}
 
 template <bool B_MN, typename OutT>
 __global__ void __launch_bounds__(kWideThreads, 1)
     gemm_relu_wide_kernel(const __grid_constant__ CUtensorMap tmA,
-                          const __grid_constant__ CUtensorMap tmB, const GemmParams p)
+                          const __grid_constant__ CUtensorMap tmB,
+                          const __grid_constant__ CUtensorMap tmC, const GemmParams p)
 {
     using Cfg = WideCfg;
     constexpr int kStages = Cfg::kStages;
@@ -79,6 +122,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     if (warp == 0 && lane == 0) {
         prefetch_tensor_map(&tmA);
         prefetch_tensor_map(&tmB);
+        if (p.c_tma) prefetch_tensor_map(&tmC);
     }
     if (warp == 1) {
         tmem_alloc<2>(smem_addr(&tmem_slot), kTmemCols);
@@ -247,11 +291,16 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         // ------------------------------------------------ epilogue (warps 2..9)
         const int q = warp & 3;          // TMEM lane quarter this warp may access
         const int g = (warp - 2) >> 2;   // which 128 columns of each half
+        constexpr bool k16 = !std::is_same_v<OutT, float>;
+        const uint32_t out_stage = tiles_base + static_cast<uint32_t>(kStages * Cfg::kStageBytes) +
+                                   static_cast<uint32_t>((warp - 2) * Cfg::kOutWarpBytes);
+        uint32_t nstore = 0;  // boxes sent so far (alternates the 16-bit staging buffers)
         int local = 0;
         for (int u = cluster_id; u < p.num_units && !aborted; u += num_clusters, ++local) {
             const WorkUnit w = decode_unit(u, p.tiles_m, p.tiles_n, 1, p.kblocks, p.panel);
             const uint32_t tphase = static_cast<uint32_t>(local) & 1u;
-            const int row = w.m_tile * Cfg::kTileM + static_cast<int>(rank) * kBM + q * 32 + lane;
+            const int row0 = w.m_tile * Cfg::kTileM + static_cast<int>(rank) * kBM + q * 32;
+            const int row = row0 + lane;
             const bool row_ok = row < p.M;
             OutT *rowp = reinterpret_cast<OutT *>(p.C) + static_cast<int64_t>(row) * p.ldc;
             for (int h = 0; h < 2; ++h) {
@@ -269,16 +318,39 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                     uint32_t v[32];
                     tmem_load_32cols(taddr + static_cast<uint32_t>(c), v);
                     tmem_load_wait();
-                    const int valid = min(32, p.N - (col0 + c));
-                    if (row_ok)
-                        store_row32<OutT>(rowp + col0 + c, v, valid, p.vec_ok != 0, p.relu,
-                                          p.c_stream != 0);
+                    if (p.c_tma) {
+                        const uint32_t box = out_stage + (k16 ? (nstore & 1u) * 2048u : 0u);
+                        // the store that last read this box has finished reading it
+                        if (lane == 0) {
+                            if constexpr (k16)
+                                bulk_wait_group_read<1>();
+                            else
+                                bulk_wait_group_read<0>();
+                        }
+                        __syncwarp();
+                        stage_row32<OutT>(box, lane, v, p.relu);
+                        fence_proxy_async_shared();
+                        __syncwarp();
+                        if (lane == 0 && row0 < p.M) {
+                            tma_store_2d(&tmC, box, col0 + c, row0);
+                            bulk_commit_group();
+                        }
+                        ++nstore;
+                    } else {
+                        const int valid = min(32, p.N - (col0 + c));
+                        if (row_ok)
+                            store_row32<OutT>(rowp + col0 + c, v, valid, p.vec_ok != 0, p.relu,
+                                              p.c_stream != 0);
+                    }
                 }
                 tc_fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive_cluster(map_shared_to_rank(smem_addr(&tempty_bar[h]), 0));
             }
         }
+        // every TMA store of this warp has read its box and written C
+        if (lane == 0) bulk_wait_group<0>();
+        __syncwarp();
     }
 
     __syncwarp();
