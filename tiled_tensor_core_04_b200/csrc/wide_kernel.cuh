@@ -16,7 +16,9 @@
 //    already) before it needs half 1 back, so draining half 1 overlaps MMA
 //    work; only the drain of half 0 is exposed.
 //  * Eight epilogue warps (two per TMEM lane quarter, 128 columns of a half
-//    each) halve the drain time.
+//    each).  A warp loads its 128 columns of a half into registers with four
+//    tcgen05.ld, waits once and frees the half before it converts and stores,
+//    so the MMA warp waits only for the TMEM reads, not for the stores.
 //  * One split only (no split-K); K blocks of 64 per stage, 48 KB per stage
 //    per CTA, 4 stages.
 //  * Output through shared memory (when C's rows are 16-byte aligned): each
@@ -48,41 +50,89 @@ struct WideCfg {
     static constexpr int kSmemBytes = kStages * kStageBytes + kOutBytes + 1024;
 };
 
-// One row's 32 outputs (ReLU, rounding) into a 32 x 32 staging box laid out
-// for the TMA store: 64-byte rows with the 64-byte swizzle (16-bit outputs)
-// or 128-byte rows with the 128-byte swizzle (fp32), i.e. 16-byte chunk i of
-// row r sits at chunk i ^ ((r >> 1) & 3), resp. i ^ (r & 7).  A warp storing
-// one chunk index of 32 rows then touches every bank once per 8 lanes.
+// ReLU and rounding of one row's 32-column chunk, in place: 16-bit outputs
+// leave 16 packed words (two values each, lower column in the low half) in
+// v[0..15], fp32 leaves 32 words.
 template <typename OutT>
-__device__ __forceinline__ void stage_row32(uint32_t box, int r, const uint32_t (&v)[32], int relu)
+__device__ __forceinline__ void finish_chunk(uint32_t (&v)[32], int relu)
 {
-    float f[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        const float x = __uint_as_float(v[i]);
-        f[i] = relu ? fmaxf(x, 0.0f) : x;
-    }
     if constexpr (std::is_same_v<OutT, float>) {
-        const uint32_t row = box + static_cast<uint32_t>(r) * 128u;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const uint32_t chunk = static_cast<uint32_t>(i ^ (r & 7));
-            st_shared_v4(row + chunk * 16u, __float_as_uint(f[4 * i]), __float_as_uint(f[4 * i + 1]),
-                         __float_as_uint(f[4 * i + 2]), __float_as_uint(f[4 * i + 3]));
+        for (int i = 0; i < 32; ++i) {
+            const float x = __uint_as_float(v[i]);
+            v[i] = __float_as_uint(relu ? fmaxf(x, 0.0f) : x);
         }
     } else {
-        const uint32_t row = box + static_cast<uint32_t>(r) * 64u;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const uint32_t chunk = static_cast<uint32_t>(i ^ ((r >> 1) & 3));
-            st_shared_v4(row + chunk * 16u, pack_pair<OutT>(f[8 * i], f[8 * i + 1]),
-                         pack_pair<OutT>(f[8 * i + 2], f[8 * i + 3]),
-                         pack_pair<OutT>(f[8 * i + 4], f[8 * i + 5]),
-                         pack_pair<OutT>(f[8 * i + 6], f[8 * i + 7]));
+        for (int i = 0; i < 16; ++i) {
+            float a = __uint_as_float(v[2 * i]), b = __uint_as_float(v[2 * i + 1]);
+            if (relu) {
+                a = fmaxf(a, 0.0f);
+                b = fmaxf(b, 0.0f);
+            }
+            v[i] = pack_pair<OutT>(a, b);
         }
     }
 }
 
+// One finished chunk into a 32 x 32 staging box laid out for the TMA store:
+// 64-byte rows with the 64-byte swizzle (16-bit outputs) or 128-byte rows
+// with the 128-byte swizzle (fp32), i.e. 16-byte piece i of row r sits at
+// piece i ^ ((r >> 1) & 3), resp. i ^ (r & 7).  A warp storing one piece
+// index of 32 rows then touches every bank once per 8 lanes.
+template <typename OutT>
+__device__ __forceinline__ void stage_chunk(uint32_t box, int r, const uint32_t (&v)[32])
+{
+    if constexpr (std::is_same_v<OutT, float>) {
+        const uint32_t row = box + static_cast<uint32_t>(r) * 128u;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            st_shared_v4(row + static_cast<uint32_t>(i ^ (r & 7)) * 16u, v[4 * i], v[4 * i + 1],
+                         v[4 * i + 2], v[4 * i + 3]);
+    } else {
+        const uint32_t row = box + static_cast<uint32_t>(r) * 64u;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            st_shared_v4(row + static_cast<uint32_t>(i ^ ((r >> 1) & 3)) * 16u, v[4 * i],
+                         v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    }
+}
+
+// One finished chunk straight to global memory (C not 16-byte aligned, or
+// evict-first stores asked for); `valid` of the 32 columns are in range.
+template <typename OutT>
+__device__ __forceinline__ void store_chunk(OutT *dst, const uint32_t (&v)[32], int valid, bool vec,
+                                            bool stream)
+{
+    constexpr int kWords = std::is_same_v<OutT, float> ? 32 : 16;
+    if (vec && valid >= 32) {
+        uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+        for (int i = 0; i < kWords / 4; ++i) {
+            const uint4 q = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            if (stream)
+                __stcs(d4 + i, q);
+            else
+                d4[i] = q;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            if (i < valid) {
+                if constexpr (std::is_same_v<OutT, float>) {
+                    dst[i] = __uint_as_float(v[i]);
+                } else {
+                    const uint16_t bits = static_cast<uint16_t>(v[i >> 1] >> (16 * (i & 1)));
+                    reinterpret_cast<uint16_t *>(dst)[i] = bits;
+                }
+            }
+        }
+    }
+}
+
+// 10 warps: three share one SM sub-partition's 16 K registers, so at most
+// 168 registers per thread; the epilogue holds 128 accumulator columns per
+// thread at once.
 template <bool B_MN, typename OutT>
 __global__ void __launch_bounds__(kWideThreads, 1)
     gemm_relu_wide_kernel(const __grid_constant__ CUtensorMap tmA,
@@ -312,12 +362,23 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                 const int col0 = w.n_tile * Cfg::kTileN + h * kBN + g * (kBN / 2);
                 const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                        static_cast<uint32_t>(h * kBN + g * (kBN / 2));
-#pragma unroll 1
-                for (int c = 0; c < kBN / 2; c += 32) {
+                // all of this warp's 128 columns of the half into registers at
+                // once, then the half goes back to the MMA warp before any store
+                constexpr int kChunks = kBN / 2 / 32;
+                uint32_t v[kChunks][32];
+#pragma unroll
+                for (int j = 0; j < kChunks; ++j)
+                    if (col0 + 32 * j < p.N) tmem_load_32cols(taddr + static_cast<uint32_t>(32 * j), v[j]);
+                tmem_load_wait();
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(map_shared_to_rank(smem_addr(&tempty_bar[h]), 0));
+#pragma unroll
+                for (int j = 0; j < kChunks; ++j) finish_chunk<OutT>(v[j], p.relu);
+#pragma unroll
+                for (int j = 0; j < kChunks; ++j) {
+                    const int c = 32 * j;
                     if (col0 + c >= p.N) break;  // warp-uniform
-                    uint32_t v[32];
-                    tmem_load_32cols(taddr + static_cast<uint32_t>(c), v);
-                    tmem_load_wait();
                     if (p.c_tma) {
                         const uint32_t box = out_stage + (k16 ? (nstore & 1u) * 2048u : 0u);
                         // the store that last read this box has finished reading it
@@ -328,7 +389,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                                 bulk_wait_group_read<0>();
                         }
                         __syncwarp();
-                        stage_row32<OutT>(box, lane, v, p.relu);
+                        stage_chunk<OutT>(box, lane, v[j]);
                         fence_proxy_async_shared();
                         __syncwarp();
                         if (lane == 0 && row0 < p.M) {
@@ -339,13 +400,10 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                     } else {
                         const int valid = min(32, p.N - (col0 + c));
                         if (row_ok)
-                            store_row32<OutT>(rowp + col0 + c, v, valid, p.vec_ok != 0, p.relu,
+                            store_chunk<OutT>(rowp + col0 + c, v[j], valid, p.vec_ok != 0,
                                               p.c_stream != 0);
                     }
                 }
-                tc_fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(map_shared_to_rank(smem_addr(&tempty_bar[h]), 0));
             }
         }
         // every TMA store of this warp has read its box and written C
