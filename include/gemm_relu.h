@@ -94,11 +94,13 @@ typedef struct {
                             and cta_pair auto), 1 = use it (needs M <= 128), 2 = never     */
     int stream_k;        /* skinny kernel: 1 = spread the K blocks of all column tiles
                             evenly over the CTAs (stream-K) instead of split-K; 0 = off  */
-    int wide;            /* CTA-pair tile of 256 x 512 (two N = 256 MMAs per K step, one
-                            TMEM accumulator released in halves): 0 = auto (when it needs
-                            no more waves of tiles than 256 x 256 does, with no split-K
-                            and stage_k unset), 1 = use it whenever the CTA pair runs
-                            without split-K, 2 = never                                    */
+    int wide;            /* CTA-pair tiles of 256 x 512 (two N = 256 MMAs per K step) or,
+                            with trans_b, 256 x 448 (two N = 224 MMAs); one TMEM
+                            accumulator released in halves.  0 = auto (the tiling with
+                            the fewest waves x work per unit, wider on ties; needs no
+                            split-K and stage_k unset), 1 = 256 x 512 whenever the CTA
+                            pair runs without split-K, 2 = never, 3 = 256 x 448 (256 x 512
+                            when B is not K-major)                                        */
 } gemm_relu_options_t;
 /* cta_pair: 0 = auto, 1 = force the 2-CTA (256 x 256 or 256 x 512 tile,
  * cta_group::2) kernel, 2 = force the 1-CTA (128 x 256 tile) kernel.  Split-K
@@ -110,7 +112,7 @@ typedef struct {
 /* What a call will do (filled by gemm_relu_plan). */
 typedef struct {
     int cta_pair;        /* 1 = 2-CTA cluster kernel, 0 = 1-CTA kernel                   */
-    int tile_m, tile_n, tile_k; /* tile_n == 512: the wide CTA-pair kernel               */
+    int tile_m, tile_n, tile_k; /* tile_n 512 or 448: the wide CTA-pair kernel           */
     int tiles_m, tiles_n;
     int kblocks;         /* ceil(K / tile_k)                                              */
     int split_k;         /* K splits per output tile (1 = none)                           */

@@ -70,11 +70,15 @@ def test_plans_for_the_workloads(lib):
     assert (p["tile_n"], p["tile_k"], p["kblocks"], p["stages"]) == (256, 128, 64, 3)
     assert (p["tiles_m"], p["tiles_n"], p["units"], p["grid_ctas"]) == (32, 32, 1024, 148)
 
-    # 14 wide columns would need 7 waves (= 14 of 256 x 256), 28 narrow ones 13
+    # N = 7168 = 16 x 448: 512 units of 256 x 448 in 7 waves (cost 7 x 1.75 = 12.25)
+    # beat 13 waves of 256 x 256 and 7 waves of 256 x 512 (cost 14)
     p = plan(wl.WORKLOADS["bt8192x7168x8192_bf16_f32"])
-    assert p["cta_pair"] == 1 and p["tile_n"] == 256 and p["tiles_n"] == 28 and p["units"] == 896
+    assert p["cta_pair"] == 1 and p["tile_n"] == 448 and p["tiles_n"] == 16 and p["units"] == 512
+    assert (p["tile_k"], p["kblocks"], p["stages"]) == (64, 128, 4)
     p = plan(wl.WORKLOADS["bt8192x7168x8192_bf16_f32"], wide=1)
     assert p["tile_n"] == 512 and p["tiles_n"] == 14 and p["units"] == 448
+    p = plan(wl.WORKLOADS["bt8192x7168x8192_bf16_f32"], wide=2)
+    assert p["tile_n"] == 256 and p["tiles_n"] == 28 and p["units"] == 896
 
     p = plan(wl.WORKLOADS["tail5000x3001x2050_f16"])
     assert p["pack_a"] == 1 and p["pack_b"] == 1          # 4100- and 6002-byte row pitches
@@ -122,8 +126,10 @@ def test_options_override_the_plan(lib):
     assert plan(w, split_k=2, wide=1)["tile_n"] == 256       # no split-K on the wide kernel
     assert plan(w, cta_pair=g.GEMM_CTA_SINGLE, wide=1)["tile_n"] == 256
     assert plan(w, stage_k=128)["tile_n"] == 256
+    assert plan(w, wide=3)["tile_n"] == 512                  # 448 needs a K-major B
+    assert g.gemm_relu_plan(4096, 4096, 4096, 0, 0, 1, options={"wide": 3})["tile_n"] == 448
     with pytest.raises(g.GemmError):
-        plan(w, wide=3)
+        plan(w, wide=4)
     assert plan(w, cta_pair=g.GEMM_CTA_SINGLE, stage_k=128)["tile_k"] == 64   # 1-CTA: 64 only
     with pytest.raises(g.GemmError):
         plan(w, stage_k=96)

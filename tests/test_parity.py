@@ -108,6 +108,10 @@ VARIANTS = {
     "wide_few": {"cta_pair": g.GEMM_CTA_PAIR, "wide": 1, "max_ctas": 4, "panel": 3},
     # evict-first stores: the wide kernel's direct (non-TMA) epilogue
     "wide_direct": {"cta_pair": g.GEMM_CTA_PAIR, "wide": 1, "c_streaming": 1},
+    # 256 x 448 tiles (two N = 224 MMAs) when B is K-major, 256 x 512 otherwise
+    "wide448": {"cta_pair": g.GEMM_CTA_PAIR, "wide": 3},
+    "wide448_few": {"cta_pair": g.GEMM_CTA_PAIR, "wide": 3, "max_ctas": 4, "panel": 3},
+    "wide448_direct": {"cta_pair": g.GEMM_CTA_PAIR, "wide": 3, "c_streaming": 1},
     "no_wide": {"wide": 2},
 }
 
@@ -123,7 +127,8 @@ def test_shapes_fp16(M, N, K, trans_b, variant):
 @pytest.mark.parametrize("in_dtype", [F16, BF16])
 @pytest.mark.parametrize("trans_b", [False, True])
 @pytest.mark.parametrize("relu", [True, False])
-@pytest.mark.parametrize("variant", ["auto", "single", "split3", "pair_k64"])
+@pytest.mark.parametrize("variant", ["auto", "single", "split3", "pair_k64", "wide", "wide_direct",
+                                     "wide448", "wide448_direct"])
 def test_dtypes_and_relu(in_dtype, out_dtype, trans_b, relu, variant):
     full_case(300, 520, 330, in_dtype, out_dtype, trans_b, relu, VARIANTS[variant], seed=7,
               dist="normal")
@@ -191,6 +196,7 @@ def test_full_size_workloads_sampled(name):
 
 @pytest.mark.parametrize("name,opt", [("square8192_f16", "no_wide"),
                                       ("bt8192x7168x8192_bf16_f32", "wide"),
+                                      ("bt8192x7168x8192_bf16_f32", "no_wide"),
                                       ("tail5000x3001x2050_f16", "no_wide")])
 def test_full_size_workloads_other_tile(name, opt):
     # the tile shape the planner did not pick for this workload
@@ -202,7 +208,8 @@ def test_full_size_workloads_other_tile(name, opt):
 
 
 # ---------------------------------------------------------------- closed forms
-@pytest.mark.parametrize("variant", ["auto", "single", "split3", "pair_k64", "wide", "wide_few"])
+@pytest.mark.parametrize("variant", ["auto", "single", "split3", "pair_k64", "wide", "wide_few",
+                                     "wide448", "wide448_few"])
 @pytest.mark.parametrize("trans_b", [False, True])
 @pytest.mark.parametrize("M,N,K", [(300, 520, 2050), (256, 512, 8192), (70, 33, 9)])
 def test_ones_give_exactly_K(M, N, K, trans_b, variant):
@@ -232,7 +239,7 @@ def test_all_negative_product_is_zero(trans_b):
 
 
 @pytest.mark.parametrize("variant", ["auto", "single", "split3", "packed", "pair_k64", "wide",
-                                     "no_wide"])
+                                     "no_wide", "wide448"])
 @pytest.mark.parametrize("trans_b", [False, True])
 @pytest.mark.parametrize("in_dtype", [F16, BF16])
 @pytest.mark.parametrize("M,N,K", [(300, 520, 1000), (129, 264, 72), (5000 // 8, 3001, 2050)])
@@ -263,7 +270,7 @@ def test_M_or_N_zero_is_a_no_op():
     assert (C.float() == 7).all()
 
 
-@pytest.mark.parametrize("variant", ["auto", "wide"])
+@pytest.mark.parametrize("variant", ["auto", "wide", "wide448"])
 @pytest.mark.parametrize("c_offset,a_offset", [(1, 0), (0, 1), (3, 5)])
 def test_misaligned_pointers(c_offset, a_offset, variant):
     full_case(260, 264, 136, F16, F16, False, options=VARIANTS[variant], c_offset=c_offset,

@@ -78,25 +78,31 @@ int variant_index(bool pair, int kk, bool b_mn, gemm_dtype_t out)
     return shape * 6 + (b_mn ? 3 : 0) + static_cast<int>(out);
 }
 
-// Wide CTA-pair kernels (256 x 512 tiles): B MN- or K-major, three output
-// types; the third tensor map describes C for the TMA-store epilogue.
+// Wide CTA-pair kernels: 256 x 512 tiles (B MN- or K-major) and 256 x 448
+// tiles (B K-major), three output types; the third tensor map describes C
+// for the TMA-store epilogue.
 using WideKernelFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
                               const GemmParams);
 
-template <bool BMN>
+template <bool BMN, int BNH>
 WideKernelFn pick_wide_out(gemm_dtype_t out)
 {
     switch (out) {
-    case GEMM_F16: return gemm_relu_wide_kernel<BMN, __half>;
-    case GEMM_BF16: return gemm_relu_wide_kernel<BMN, __nv_bfloat16>;
-    default: return gemm_relu_wide_kernel<BMN, float>;
+    case GEMM_F16: return gemm_relu_wide_kernel<BMN, __half, BNH>;
+    case GEMM_BF16: return gemm_relu_wide_kernel<BMN, __nv_bfloat16, BNH>;
+    default: return gemm_relu_wide_kernel<BMN, float, BNH>;
     }
 }
 
-WideKernelFn pick_wide(bool b_mn, gemm_dtype_t out)
+// bnh: MMA half width (tile_n / 2), 256 or 224 (224 with b_mn == false only)
+WideKernelFn pick_wide(bool b_mn, int bnh, gemm_dtype_t out)
 {
-    return b_mn ? pick_wide_out<true>(out) : pick_wide_out<false>(out);
+    if (bnh == 224) return pick_wide_out<false, 224>(out);
+    return b_mn ? pick_wide_out<true, 256>(out) : pick_wide_out<false, 256>(out);
 }
+
+int wide_smem(int bnh) { return bnh == 224 ? WideCfg<224>::kSmemBytes : WideCfg<256>::kSmemBytes; }
+int wide_stages(int bnh) { return bnh == 224 ? WideCfg<224>::kStages : WideCfg<256>::kStages; }
 
 // Skinny-M (swap-AB) kernels: NP in {16, 32, 64, 128}, B MN- or K-major.
 template <int NP, bool BMN>
@@ -160,7 +166,7 @@ struct DeviceInfo {
     int max_pair_clusters = 0;
     bool attr_set[18] = {};
     bool skinny_attr_set[24] = {};
-    bool wide_attr_set[6] = {};
+    bool wide_attr_set[9] = {};
 };
 
 std::mutex g_dev_mutex;
@@ -190,13 +196,12 @@ gemm_status_t ensure_skinny_attr(DeviceInfo &d, int np, bool b_mn, gemm_dtype_t 
     return GEMM_OK;
 }
 
-gemm_status_t ensure_wide_attr(DeviceInfo &d, bool b_mn, gemm_dtype_t out)
+gemm_status_t ensure_wide_attr(DeviceInfo &d, bool b_mn, int bnh, gemm_dtype_t out)
 {
-    const int v = (b_mn ? 3 : 0) + static_cast<int>(out);
+    const int v = (bnh == 224 ? 6 : b_mn ? 3 : 0) + static_cast<int>(out);
     if (d.wide_attr_set[v]) return GEMM_OK;
-    cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void *>(pick_wide(b_mn, out)),
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         WideCfg::kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void *>(pick_wide(b_mn, bnh, out)),
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, wide_smem(bnh));
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(wide)");
     d.wide_attr_set[v] = true;
     return GEMM_OK;
@@ -279,7 +284,7 @@ gemm_status_t make_plan(int64_t M, int64_t N, int64_t K, gemm_dtype_t in, gemm_d
     if (o.cta_pair < 0 || o.cta_pair > 2 || o.split_k < 0 || o.panel < 0 || o.max_ctas < 0 ||
         (o.stage_k != 0 && o.stage_k != 64 && o.stage_k != 128) || o.l2_hint_a < 0 ||
         o.l2_hint_a > 2 || o.l2_hint_b < 0 || o.l2_hint_b > 2 || o.c_streaming < 0 || o.c_streaming > 1 || o.swap_ab < 0 || o.swap_ab > 2 ||
-        o.stream_k < 0 || o.stream_k > 1 || o.wide < 0 || o.wide > 2)
+        o.stream_k < 0 || o.stream_k > 1 || o.wide < 0 || o.wide > 3)
         return GEMM_ERR_INVALID_ARG;
 
     gemm_relu_plan_t p = {};
@@ -364,25 +369,35 @@ gemm_status_t make_plan(int64_t M, int64_t N, int64_t K, gemm_dtype_t in, gemm_d
     int64_t clusters = max_pair_clusters > 0 ? max_pair_clusters : num_sms / 2;
     if (o.max_ctas > 0) clusters = std::min<int64_t>(clusters, std::max(1, o.max_ctas / 2));
     clusters = std::max<int64_t>(1, clusters);
-    // 256 x 512 pair tiles: half the units, each twice the work; taken when
-    // that costs no more waves of units than 256 x 256 tiles
-    bool wide = false;
+    // Pair tiles of 256 x 512 (or 256 x 448 when B is K-major) do 2 (1.75)
+    // times the work of a 256 x 256 unit with fewer operand bytes per flop.
+    // Cost of a tiling = waves of units x work per unit; the cheapest wins,
+    // ties going to the wider tile.
+    int wide_n = 0;  // 0, 512 or 448
     if (pair && split == 1 && o.wide != 2) {
         if (o.wide == 1)
-            wide = true;
+            wide_n = 2 * kBN;
+        else if (o.wide == 3)
+            wide_n = trans_b ? 448 : 2 * kBN;
         else if (o.stage_k == 0) {
-            const int64_t waves_sq = ceil_div(tiles_m * tiles_n, clusters);
-            const int64_t waves_wide = ceil_div(tiles_m * ceil_div(N, 2 * kBN), clusters);
-            wide = 2 * waves_wide <= waves_sq;
+            const int64_t cost_sq = 8 * ceil_div(tiles_m * tiles_n, clusters);
+            const int64_t cost_512 = 16 * ceil_div(tiles_m * ceil_div(N, 512), clusters);
+            const int64_t cost_448 = trans_b ? 14 * ceil_div(tiles_m * ceil_div(N, 448), clusters)
+                                             : INT64_MAX;
+            if (cost_512 <= cost_sq && cost_512 <= cost_448)
+                wide_n = 512;
+            else if (cost_448 <= cost_sq)
+                wide_n = 448;
         }
     }
+    const bool wide = wide_n > 0;
     // the 256 x 256 pair kernel takes 128 of K per pipeline stage unless asked
     // for 64; the wide kernel takes 64
     const int kk = (pair && !wide && o.stage_k != 64) ? 2 : 1;
     p.tile_k = kBK * kk;
     p.kblocks = static_cast<int>(ceil_div(K, p.tile_k));
-    if (wide) p.tile_n = 2 * kBN;
-    const int64_t tiles_n_used = wide ? ceil_div(N, 2 * kBN) : tiles_n;
+    if (wide) p.tile_n = wide_n;
+    const int64_t tiles_n_used = wide ? ceil_div(N, wide_n) : tiles_n;
     const int64_t units = tiles_m * tiles_n_used * split;
     if (units > INT32_MAX) return GEMM_ERR_INVALID_ARG;
     p.tiles_m = static_cast<int>(tiles_m);
@@ -391,7 +406,7 @@ gemm_status_t make_plan(int64_t M, int64_t N, int64_t K, gemm_dtype_t in, gemm_d
     p.panel = o.panel > 0 ? o.panel : kDefaultPanel;
     if (p.tiles_m > 0) p.panel = std::min(p.panel, p.tiles_m);
     p.units = static_cast<int>(units);
-    p.stages = wide ? WideCfg::kStages : stage_count(pair, kk);
+    p.stages = wide ? wide_stages(wide_n / 2) : stage_count(pair, kk);
 
     int64_t grid;
     if (pair) {
@@ -745,7 +760,10 @@ gemm_status_t run(const void *A, const void *B, void *C, int64_t M, int64_t N, i
     const bool pair = plan.cta_pair != 0;
     const int kk = plan.tile_k / kBK;
     const bool b_mn = !trans_b;
-    const int bn_cta = pair ? kBN / 2 : kBN;
+    const bool wide = plan.tile_n > kBN;
+    const int bnh = plan.tile_n / 2;  // wide kernels: MMA half width
+    // rows of a K-major B box: this CTA's share of one MMA's N
+    const int bn_cta = wide ? bnh / 2 : pair ? kBN / 2 : kBN;
     CUtensorMap tmA, tmB;
     st = encode_2d(&tmA, a_src, in, K, M, a_pitch, kBK, kBM);
     if (st != GEMM_OK) return st;
@@ -772,14 +790,13 @@ gemm_status_t run(const void *A, const void *B, void *C, int64_t M, int64_t N, i
     p.num_units = plan.units;
     p.relu = split ? 0 : (relu ? 1 : 0);
     p.vec_ok = (!misaligned16(p.C) && ((N * static_cast<int64_t>(dtype_size(kout))) % 16) == 0) ? 1 : 0;
-    p.idesc = make_idesc(in, b_mn, pair ? 2 * kBM : kBM, kBN);
+    p.idesc = make_idesc(in, b_mn, pair ? 2 * kBM : kBM, wide ? bnh : kBN);
     p.timeout_ns = (opts && opts->timeout_ns) ? opts->timeout_ns : kDefaultTimeoutNs;
     p.l2_a = opts ? opts->l2_hint_a : 0;
     p.l2_b = opts ? opts->l2_hint_b : 0;
     p.c_stream = (!split && opts) ? opts->c_streaming : 0;
     p.sleep_ns = (opts && opts->wait_sleep_ns) ? opts->wait_sleep_ns : 0;
 
-    const bool wide = plan.tile_n == WideCfg::kTileN;
     // the wide kernel writes C with TMA stores of 32 x 32 boxes when C's base
     // and row pitch are 16-byte aligned (what a tensor map needs) and no
     // evict-first stores were asked for
@@ -792,14 +809,14 @@ gemm_status_t run(const void *A, const void *B, void *C, int64_t M, int64_t N, i
     }
     {
         std::lock_guard<std::mutex> lock(g_dev_mutex);
-        st = wide ? ensure_wide_attr(*dev, b_mn, kout) : ensure_kernel_attr(*dev, pair, kk, b_mn, kout);
+        st = wide ? ensure_wide_attr(*dev, b_mn, bnh, kout) : ensure_kernel_attr(*dev, pair, kk, b_mn, kout);
     }
     if (st != GEMM_OK) return st;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(plan.grid_ctas), 1, 1);
     cfg.blockDim = dim3(wide ? kWideThreads : kThreads, 1, 1);
-    cfg.dynamicSmemBytes = wide ? WideCfg::kSmemBytes : smem_bytes(pair, kk);
+    cfg.dynamicSmemBytes = wide ? wide_smem(bnh) : smem_bytes(pair, kk);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -808,7 +825,7 @@ gemm_status_t run(const void *A, const void *B, void *C, int64_t M, int64_t N, i
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pair ? 1 : 0;
-    cudaError_t e = wide ? cudaLaunchKernelEx(&cfg, pick_wide(b_mn, kout), tmA, tmB, tmC, p)
+    cudaError_t e = wide ? cudaLaunchKernelEx(&cfg, pick_wide(b_mn, bnh, kout), tmA, tmB, tmC, p)
                          : cudaLaunchKernelEx(&cfg, pick_kernel(pair, kk, b_mn, kout), tmA, tmB, p);
     if (e != cudaSuccess) return cuda_fail(e, "gemm kernel launch");
 

@@ -1,14 +1,16 @@
-// wide_kernel.cuh -- the 256 x 512 CTA-pair variant of the fused GEMM + ReLU
+// wide_kernel.cuh -- the 256 x 512 (and 256 x 448) CTA-pair variant of the fused GEMM + ReLU
 // tile loop (the "Tiled GEMM with a fused ReLU epilogue" example of the
 // TileLang notes, T.gemm into a fragment accumulator, T.max(C, 0) on the way
 // out, computed here with tcgen05 tensor cores).
 //
 // Same roles, barriers and bounded waits as gemm_kernel.cuh; what differs:
-//  * One unit is a 256 x 512 tile of C.  Each CTA of the pair holds 128 rows
-//    of A and 256 of the tile's columns of B (128 of each 256-column half);
-//    every K step issues two cta_group::2 MMAs of M = 256, N = 256, one per
-//    half.  Per flop, the pair reads 25 % fewer operand bytes from L2 than a
-//    256 x 256 tile, and one wave of tiles touches fewer DRAM bytes.
+//  * One unit is a 256 x 2*BNH tile of C (BNH = 256, or 224 when B is
+//    K-major).  Each CTA of the pair holds 128 rows of A and BNH of the
+//    tile's columns of B (BNH / 2 of each half); every K step issues two
+//    cta_group::2 MMAs of M = 256, N = BNH, one per half.  Per flop, a 256 x
+//    512 tile reads 25 % fewer operand bytes from L2 than a 256 x 256 tile,
+//    and one wave of tiles touches fewer DRAM bytes.  The 448-column tile
+//    covers N = 7168 in 16 whole tiles.
 //  * The fp32 accumulator fills all 512 TMEM columns, so there is a single
 //    accumulator, released in two 256-column halves: the epilogue drains
 //    half 0, frees it, then half 1.  At the start of a unit the MMA warp
@@ -35,19 +37,30 @@ namespace gr {
 constexpr int kWideThreads = 320;  // producer, MMA, 8 epilogue warps
 constexpr int kWideEpiWarps = 8;
 
+// BNH: columns of one MMA half (the MMA's N): 256, or 224 for B stored
+// K-major only (each CTA then holds 112 rows of B per half; 112 columns do
+// not split into the 64-column boxes of an MN-major B).
+template <int BNH>
 struct WideCfg {
+    static_assert(BNH == 256 || BNH == 224, "MMA halves of 256 or 224 columns");
     static constexpr int kTileM = 2 * kBM;                  // 256 rows per CTA pair
-    static constexpr int kTileN = 2 * kBN;                  // 512 columns: two MMA halves
+    static constexpr int kTileN = 2 * BNH;                  // two MMA halves
+    static constexpr int kBRows = BNH / 2;                  // B columns per CTA and half
     static constexpr int kABytes = kBM * kBK * 2;           // 16 KB: 128 rows x 64 K
-    static constexpr int kBHalf = (kBN / 2) * kBK * 2;      // 16 KB: 128 columns x 64 K
-    static constexpr int kStageBytes = kABytes + 2 * kBHalf;  // 48 KB
-    static constexpr int kStagesFit = (232448 - 2048) / kStageBytes;
+    static constexpr int kBHalf = kBRows * kBK * 2;         // 16 or 14 KB
+    static constexpr int kStageBytes = kABytes + 2 * kBHalf;  // 48 or 44 KB
+    static constexpr int kOutWarpBytes = 4096;  // one 32 x 32 fp32 box or two 16-bit boxes
+    static constexpr int kOutBytes = kWideEpiWarps * kOutWarpBytes;
+    // stages that fit in 227 KB next to the staging boxes, 1 KB of static
+    // shared memory and 1 KB of alignment slack
+    static constexpr int kStagesFit = (232448 - 2048 - kOutBytes) / kStageBytes;
     static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
     // the loads of both CTAs complete on the leader's barrier
     static constexpr uint32_t kTxBytes = 2 * kStageBytes;
-    static constexpr int kOutWarpBytes = 4096;  // one 32 x 32 fp32 box or two 16-bit boxes
-    static constexpr int kOutBytes = kWideEpiWarps * kOutWarpBytes;
     static constexpr int kSmemBytes = kStages * kStageBytes + kOutBytes + 1024;
+    // 32-column chunks of one half drained by epilogue warp group g (128 + the rest)
+    static constexpr int kChunksG0 = 4;
+    static constexpr int kChunksG1 = (BNH - 128) / 32;
 };
 
 // ReLU and rounding of one row's 32-column chunk, in place: 16-bit outputs
@@ -133,13 +146,14 @@ __device__ __forceinline__ void store_chunk(OutT *dst, const uint32_t (&v)[32], 
 // 10 warps: three share one SM sub-partition's 16 K registers, so at most
 // 168 registers per thread; the epilogue holds 128 accumulator columns per
 // thread at once.
-template <bool B_MN, typename OutT>
+template <bool B_MN, typename OutT, int BNH>
 __global__ void __launch_bounds__(kWideThreads, 1)
     gemm_relu_wide_kernel(const __grid_constant__ CUtensorMap tmA,
                           const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ CUtensorMap tmC, const GemmParams p)
 {
-    using Cfg = WideCfg;
+    using Cfg = WideCfg<BNH>;
+    static_assert(!B_MN || BNH == 256, "MN-major B needs 256-column halves");
     constexpr int kStages = Cfg::kStages;
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -201,7 +215,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
             for (int u = cluster_id; u < p.num_units && !aborted; u += num_clusters, ++local) {
                 const WorkUnit w = decode_unit(u, p.tiles_m, p.tiles_n, 1, p.kblocks, p.panel);
                 const int m_row = w.m_tile * Cfg::kTileM + static_cast<int>(rank) * kBM;
-                const int n_col = w.n_tile * Cfg::kTileN + static_cast<int>(rank) * (kBN / 2);
+                const int n_col = w.n_tile * Cfg::kTileN + static_cast<int>(rank) * Cfg::kBRows;
                 for (int i = 0; i < w.kb1 - w.kb0; ++i) {
                     const int kb = k_block_at(w, i, local);
                     if (!wait_phase_thread<false>(smem_addr(&empty_bar[stage]), phase ^ 1u, wc,
@@ -218,7 +232,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                     tma_load_2d_pair_hint(a_dst, &tmA, fb_leader, kx, m_row, pol_a);
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
-                        const int n = n_col + h * kBN;
+                        const int n = n_col + h * BNH;
                         const uint32_t dst = b_dst + static_cast<uint32_t>(h * Cfg::kBHalf);
                         if constexpr (B_MN) {
                             tma_load_2d_pair_hint(dst, &tmB, fb_leader, n, kx, pol_b);
@@ -261,6 +275,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
             // four K = 16 MMAs of one stage into accumulator half h
             auto issue_half = [&](int s, int h, bool first) {
                 const uint64_t so = static_cast<uint64_t>(s) * kStageStep;
+                // half h accumulates at TMEM column 256 * h (for BNH = 224 too)
                 const uint32_t d = tmem_base + static_cast<uint32_t>(h * kBN);
 #pragma unroll
                 for (int k = 0; k < kBK / 16; ++k)
@@ -359,16 +374,19 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                     break;
                 }
                 tc_fence_after_sync();
-                const int col0 = w.n_tile * Cfg::kTileN + h * kBN + g * (kBN / 2);
+                const int col0 = w.n_tile * Cfg::kTileN + h * BNH + g * 128;
                 const uint32_t taddr = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
-                                       static_cast<uint32_t>(h * kBN + g * (kBN / 2));
-                // all of this warp's 128 columns of the half into registers at
-                // once, then the half goes back to the MMA warp before any store
-                constexpr int kChunks = kBN / 2 / 32;
+                                       static_cast<uint32_t>(h * kBN + g * 128);
+                // all of this warp's columns of the half (128, or 96 for the
+                // second group of a 224-column half) into registers at once,
+                // then the half goes back to the MMA warp before any store
+                constexpr int kChunks = Cfg::kChunksG0;
+                const int nchunks = g == 0 ? Cfg::kChunksG0 : Cfg::kChunksG1;
                 uint32_t v[kChunks][32];
 #pragma unroll
                 for (int j = 0; j < kChunks; ++j)
-                    if (col0 + 32 * j < p.N) tmem_load_32cols(taddr + static_cast<uint32_t>(32 * j), v[j]);
+                    if (j < nchunks && col0 + 32 * j < p.N)
+                        tmem_load_32cols(taddr + static_cast<uint32_t>(32 * j), v[j]);
                 tmem_load_wait();
                 tc_fence_before_sync();
                 __syncwarp();
@@ -378,7 +396,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
 #pragma unroll
                 for (int j = 0; j < kChunks; ++j) {
                     const int c = 32 * j;
-                    if (col0 + c >= p.N) break;  // warp-uniform
+                    if (j >= nchunks || col0 + c >= p.N) break;  // warp-uniform
                     if (p.c_tma) {
                         const uint32_t box = out_stage + (k16 ? (nstore & 1u) * 2048u : 0u);
                         // the store that last read this box has finished reading it
