@@ -266,7 +266,9 @@ def bench_ours(args, world, rank, local):
         else:
             g.gemm_relu_ex(a, b, c, w.M, w.N, w.K, w.in_dtype, w.out_dtype, w.trans_b, w.relu,
                            sptr, options=opts)
-    launches_per_step = 1 + plan["pack_a"] + plan["pack_b"] + (1 if plan["split_k"] > 1 else 0)
+    # split-K and stream-K add their fp32 pieces in a separate reduction launch
+    launches_per_step = (1 + plan["pack_a"] + plan["pack_b"]
+                         + (1 if plan["split_k"] > 1 or plan["stream_k"] > 0 else 0))
 
     flush = None
     if (w.M * w.K + w.N * w.K) * torch.finfo(w.in_dtype).bits // 8 <= L2_BYTES:
