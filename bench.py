@@ -48,9 +48,10 @@ L2_BYTES = 126 * 2 ** 20
 # from an ncu capture, keyed by the sha256 of the kernel sources it was taken
 # on (a changed kernel reports null until it is profiled again).
 NCU_TRAFFIC_BYTES: dict[str, dict[str, float]] = {
-    # profiles/gemm_relu_tc_kernel_square8192_f16.md, profiles/gemm_relu_skinny_kernel_*.md
-    "8d47e46a261f9e96": {"square8192_f16": 825.782016e6 + 126.7008e6,
-                         "skinny64x8192x8192_f16": 135.315968e6 + 4.689664e6},
+    # profiles/gemm_relu_wide_kernel_*.md, profiles/gemm_relu_skinny_kernel_*.md
+    "52b67171c34c9af6": {"square8192_f16": 743.915264e6 + 120.3392e6,
+                         "bt8192x7168x8192_bf16_f32": 692.724736e6 + 207.65312e6,
+                         "skinny64x8192x8192_f16": 135.314432e6 + 3.935488e6},
 }
 
 _DT = {torch.float16: "f16", torch.bfloat16: "bf16", torch.float32: "f32"}
