@@ -88,6 +88,9 @@ SHAPES = [
     (1, 1, 1),           # everything re-pitched, one element
     (3, 5, 7),
     (37, 1000, 24),
+    (256, 512, 64),      # exactly one 256 x 512 tile, one K block
+    (257, 449, 130),     # one past a 256 x 448 tile; K tail of 2
+    (520, 1400, 320),    # wide tiles: ragged in M and N, 5 K blocks (more than the ring)
 ]
 
 VARIANTS = {
