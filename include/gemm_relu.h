@@ -102,9 +102,12 @@ typedef struct {
                             pair runs without split-K, 2 = never, 3 = 256 x 448 (256 x 512
                             when B is not K-major)                                        */
 } gemm_relu_options_t;
-/* cta_pair: 0 = auto, 1 = force the 2-CTA (256 x 256 or 256 x 512 tile,
- * cta_group::2) kernel, 2 = force the 1-CTA (128 x 256 tile) kernel.  Split-K
- * always uses the 1-CTA kernel. */
+/* cta_pair: 0 = auto, 1 = force a 2-CTA (cta_group::2) kernel (256 x 256,
+ * 256 x 512 or 256 x 448 tiles, see `wide`), 2 = force the 1-CTA (128 x 256
+ * tile) kernel.  Split-K always uses the 1-CTA kernel.  The wide kernels
+ * write C through shared memory with TMA stores when C's base address and row
+ * pitch are 16-byte aligned (and c_streaming is 0), with plain stores
+ * otherwise. */
 #define GEMM_CTA_AUTO 0
 #define GEMM_CTA_PAIR 1
 #define GEMM_CTA_SINGLE 2

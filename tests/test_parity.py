@@ -287,6 +287,10 @@ def test_runs_are_deterministic():
     assert torch.equal(c1, c2)
     A, B = wl.make_inputs(700, 900, 1500, F16, True, "uniform", seed=12)
     assert torch.equal(run(A, B, F32, True), run(A, B, F32, True))
+    # the wide kernels: one CTA pair per tile, serpentine K order fixed by the grid
+    for opt in ("wide", "wide448"):
+        c1 = run(A, B, F32, True, True, VARIANTS[opt])
+        assert torch.equal(c1, run(A, B, F32, True, True, VARIANTS[opt]))
 
 
 def test_side_stream_and_matmul_relu_helper():
