@@ -109,8 +109,10 @@ def small_int_inputs(M: int, N: int, K: int, in_dtype: torch.dtype, trans_b: boo
     return A, B
 
 
-def tile_boundaries(extent: int, tiles=(128, 256)) -> list[int]:
-    """Indices at tile edges for 128- and 256-wide tilings, plus the middle and the end."""
+def tile_boundaries(extent: int, tiles=(128, 224, 256, 448, 512)) -> list[int]:
+    """Indices at tile edges for the 128-, 256-, 448- and 512-wide tilings (and the 224-column
+    halves of a 448-wide tile): the first two edges and the last of each, plus the middle
+    and the end."""
     idx = {0, extent - 1, extent // 2 - 1, extent // 2}
     for t in tiles:
         for v in (t - 1, t, 2 * t - 1, 2 * t):
