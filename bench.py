@@ -258,11 +258,21 @@ def bench_ours(args, world, rank, local):
     sptr = stream.cuda_stream
     props = torch.cuda.get_device_properties(dev)
     opts = json.loads(args.options) if args.options else None
+    tuned = None
+    if args.autotune:
+        # time the candidate settings on this device first; the run then uses the fastest
+        from tiled_tensor_core_04_b200 import autotune
+        big = (w.M * w.K + w.N * w.K) * torch.finfo(w.in_dtype).bits // 8 > L2_BYTES
+        best, table = autotune.tune(A, B, C, w.M, w.N, w.K, w.in_dtype, w.out_dtype, w.trans_b,
+                                    w.relu, stream, iters=10, warmup=3,
+                                    flush_bytes=0 if big else 256 * 2 ** 20)
+        opts = best if best is not None else {}
+        tuned = {"best": best, "table": [{"options": o, "ms": ms} for o, ms in table]}
     plan = g.gemm_relu_plan(w.M, w.N, w.K, w.in_dtype, w.out_dtype, w.trans_b, A, B,
                             num_sms=props.multi_processor_count, options=opts)
 
     def call(a, b, c):
-        if opts is None:   # the plain C entry point
+        if not opts:   # the plain C entry point
             g.gemm_relu(a, b, c, w.M, w.N, w.K, w.in_dtype, w.out_dtype, w.trans_b, w.relu, sptr)
         else:
             g.gemm_relu_ex(a, b, c, w.M, w.N, w.K, w.in_dtype, w.out_dtype, w.trans_b, w.relu,
@@ -448,6 +458,7 @@ def bench_ours(args, world, rank, local):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": sampler.summary(),
         "best_of": best_of,
+        **({"autotune": tuned} if tuned is not None else {}),
         "sustained": sustained if sustained is not None else
         ("not run: L2 flush between steps" if flush is not None else "not run (--sustained-s 0)"),
         "plan": {k: plan[k] for k in ("cta_pair", "tile_m", "tile_n", "tile_k", "split_k",
@@ -472,6 +483,8 @@ def main():
     ap.add_argument("--sustained-s", type=float, default=2.0,
                     help="seconds of back-to-back calls for the 'sustained' figure (0: skip; "
                          "only when the inputs exceed L2, so no flush is needed)")
+    ap.add_argument("--autotune", action="store_true",
+                    help="time the candidate tile / hint settings first and run the fastest")
     ap.add_argument("--options", default="",
                     help='JSON object of gemm_relu_options_t fields, e.g. \'{"panel": 4}\'; '
                          "the call then goes through gemm_relu_ex")

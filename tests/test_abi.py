@@ -256,3 +256,27 @@ def test_no_device_is_reported_not_faked(lib):
     st = g.gemm_relu(0x1000, 0x2000, 0x3000, 4, 4, 4, 0, 0, 0, 1, 0, check=False)
     assert st == g.GEMM_ERR_NO_DEVICE
     assert g.gemm_relu_selftest_timeout(1000000) == g.GEMM_ERR_NO_DEVICE
+
+
+# ---------------------------------------------------------------- autotune (host logic)
+def test_autotune_candidates_are_distinct_plans(lib):
+    from tiled_tensor_core_04_b200 import autotune as at
+    for w in wl.WORKLOADS.values():
+        cands = at.candidates(w.M, w.N, w.K, w.in_dtype, w.out_dtype, w.trans_b)
+        assert cands[0] is None                      # the planner's own choice comes first
+        keys = set()
+        for o in cands:
+            p = g.gemm_relu_plan(w.M, w.N, w.K, w.in_dtype, w.out_dtype, w.trans_b, options=o)
+            knobs = {k: v for k, v in (o or {}).items() if k in at.RUNTIME_KNOBS}
+            keys.add((tuple(sorted(p.items())), tuple(sorted(knobs.items()))))
+        assert len(keys) == len(cands)               # no two candidates do the same thing
+
+
+def test_autotune_candidates_cover_the_tile_shapes(lib):
+    from tiled_tensor_core_04_b200 import autotune as at
+    tile_ns = {g.gemm_relu_plan(8192, 7168, 8192, 1, 2, True, options=o)["tile_n"]
+               for o in at.candidates(8192, 7168, 8192, 1, 2, True)}
+    assert tile_ns == {256, 448, 512}                 # K-major B: all three pair widths
+    sk = [o for o in at.candidates(64, 8192, 8192, 0, 0, False) if o and o.get("swap_ab")]
+    assert {o.get("split_k") for o in sk if "split_k" in o} >= {1, 4, 8}
+    assert any(o.get("stream_k") for o in sk)
