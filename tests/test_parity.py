@@ -109,7 +109,7 @@ VARIANTS = {
     "no_swap": {"swap_ab": 2},
     "wide": {"cta_pair": g.GEMM_CTA_PAIR, "wide": 1},
     "wide_few": {"cta_pair": g.GEMM_CTA_PAIR, "wide": 1, "max_ctas": 4, "panel": 3},
-    # evict-first stores: the wide kernel's direct (non-TMA) epilogue
+    # evict-first stores: the wide kernel's direct (16-byte vector) epilogue
     "wide_direct": {"cta_pair": g.GEMM_CTA_PAIR, "wide": 1, "c_streaming": 1},
     # 256 x 448 tiles (two N = 224 MMAs) when B is K-major, 256 x 512 otherwise
     "wide448": {"cta_pair": g.GEMM_CTA_PAIR, "wide": 3},
@@ -135,6 +135,17 @@ def test_shapes_fp16(M, N, K, trans_b, variant):
 def test_dtypes_and_relu(in_dtype, out_dtype, trans_b, relu, variant):
     full_case(300, 520, 330, in_dtype, out_dtype, trans_b, relu, VARIANTS[variant], seed=7,
               dist="normal")
+
+
+@pytest.mark.parametrize("out_dtype", [F16, BF16, F32])
+@pytest.mark.parametrize("in_dtype", [F16, BF16])
+@pytest.mark.parametrize("trans_b", [False, True])
+@pytest.mark.parametrize("variant", ["wide", "wide448"])
+def test_wide_direct_stores_all_dtypes(in_dtype, out_dtype, trans_b, variant):
+    # C one element off a 16-byte boundary: no tensor map for C and no vector
+    # stores, the wide kernels' direct epilogue runs with scalar stores
+    full_case(300, 520, 330, in_dtype, out_dtype, trans_b, True, VARIANTS[variant], seed=8,
+              dist="normal", c_offset=1)
 
 
 @pytest.mark.parametrize("variant", ["swap", "swap_split3", "swap_streamk", "swap_streamk_few",
