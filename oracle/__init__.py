@@ -34,6 +34,8 @@ _lib = None
 
 F16 = 0
 BF16 = 1
+E4M3 = 3   # torch.float8_e4m3fn
+E5M2 = 4   # torch.float8_e5m2
 
 _CFLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-fopenmp", "-fPIC", "-shared",
            "-Wall", "-Wextra"]
@@ -65,18 +67,27 @@ def _bind(path: str):
     return lib
 
 
+_FP8 = {torch.float8_e4m3fn: 3, torch.float8_e5m2: 4}
+
+
 def _code(dtype: torch.dtype) -> int:
     if dtype == torch.float16:
         return F16
     if dtype == torch.bfloat16:
         return BF16
-    raise TypeError(f"oracle inputs must be float16 or bfloat16, got {dtype}")
+    if dtype in _FP8:
+        return _FP8[dtype]
+    raise TypeError(f"oracle inputs must be float16, bfloat16, float8_e4m3fn or float8_e5m2, "
+                    f"got {dtype}")
 
 
 def _bits(t: torch.Tensor) -> np.ndarray:
-    """The raw 16-bit patterns of a CPU fp16/bf16 tensor, contiguous."""
+    """The raw bit patterns of a CPU tensor as 16-bit words, contiguous (an 8-bit
+    value goes to the low byte of its word)."""
     if t.device.type != "cpu":
         raise ValueError("oracle inputs must be CPU tensors")
+    if t.dtype in _FP8:
+        return np.ascontiguousarray(t.contiguous().view(torch.uint8).numpy()).astype(np.uint16)
     return np.ascontiguousarray(t.contiguous().view(torch.int16).numpy()).view(np.uint16)
 
 
@@ -107,7 +118,8 @@ class Oracle:
         return int(self.lib.oracle_num_threads())
 
     def decode(self, bits: np.ndarray, dtype: torch.dtype) -> np.ndarray:
-        """Widen raw fp16/bf16 bit patterns (uint16) to float64 with the oracle's decoder."""
+        """Widen raw fp16/bf16 bit patterns (uint16; fp8 patterns in the low byte) to float64
+        with the oracle's decoder."""
         src = np.ascontiguousarray(bits, dtype=np.uint16)
         out = np.empty(src.shape, dtype=np.float64)
         rc = self.lib.oracle_decode(src.ctypes.data, out.ctypes.data, src.size, _code(dtype))

@@ -34,6 +34,10 @@
  * -ffp-contract=off).  The result is returned as double, unrounded; the
  * output cast to fp16/bf16/fp32 is not applied here.
  *
+ * 8-bit floating-point inputs (E4M3, E5M2) arrive as one value per 16-bit
+ * element (the byte in the low half) and are widened exactly in the same way;
+ * their products (4+4 or 3+3 significand bits) are exact as well.
+ *
  * The loop order i-k-j used for trans_b == 0 is only a memory-order choice:
  * every output still receives its K terms one at a time in increasing k, so
  * the result is bit-identical to the textbook i-j-k triple loop.
@@ -46,7 +50,7 @@
 #include <omp.h>
 #endif
 
-enum { ORACLE_F16 = 0, ORACLE_BF16 = 1 };
+enum { ORACLE_F16 = 0, ORACLE_BF16 = 1, ORACLE_E4M3 = 3, ORACLE_E5M2 = 4 };
 
 /* IEEE-754 binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction
  * bits.  Exponent 0 encodes zero/subnormals (value = frac * 2^-24), exponent
@@ -83,15 +87,64 @@ static double decode_bf16(uint16_t h)
     return sign ? -v : v;
 }
 
+/* 8-bit E4M3 as defined by the OCP 8-bit floating point format (OFP8, the
+ * "fn" flavour): 1 sign bit, 4 exponent bits (bias 7), 3 fraction bits;
+ * exponent 0 encodes zero/subnormals (value = frac * 2^-9); there are no
+ * infinities, and only S.1111.111 is NaN (S.1111.000-110 are normal numbers,
+ * up to 448).  The value sits in the low byte of v. */
+static double decode_e4m3(uint16_t v)
+{
+    int sign = (v >> 7) & 1;
+    int expo = (v >> 3) & 0xf;
+    int frac = v & 0x7;
+    double x;
+    if (expo == 0xf && frac == 0x7)
+        x = NAN;
+    else if (expo == 0)
+        x = ldexp((double)frac, -9);
+    else
+        x = ldexp((double)(frac | 0x8), expo - 10);
+    return sign ? -x : x;
+}
+
+/* 8-bit E5M2 (OFP8): 1 sign bit, 5 exponent bits (bias 15), 2 fraction bits,
+ * IEEE-like: exponent 0 gives zero/subnormals (frac * 2^-16), exponent 31
+ * infinity (frac == 0) or NaN.  The value sits in the low byte of v. */
+static double decode_e5m2(uint16_t v)
+{
+    int sign = (v >> 7) & 1;
+    int expo = (v >> 2) & 0x1f;
+    int frac = v & 0x3;
+    double x;
+    if (expo == 0)
+        x = ldexp((double)frac, -16);
+    else if (expo == 31)
+        x = frac ? NAN : INFINITY;
+    else
+        x = ldexp((double)(frac | 0x4), expo - 17);
+    return sign ? -x : x;
+}
+
+static double decode_one(uint16_t v, int dtype)
+{
+    switch (dtype) {
+    case ORACLE_F16: return decode_f16(v);
+    case ORACLE_BF16: return decode_bf16(v);
+    case ORACLE_E4M3: return decode_e4m3(v);
+    default: return decode_e5m2(v);
+    }
+}
+
+static int valid_dtype(int dtype)
+{
+    return dtype == ORACLE_F16 || dtype == ORACLE_BF16 || dtype == ORACLE_E4M3 ||
+           dtype == ORACLE_E5M2;
+}
+
 static int decode_array(const uint16_t *src, double *dst, int64_t n, int dtype)
 {
-    if (dtype == ORACLE_F16) {
-        for (int64_t i = 0; i < n; ++i) dst[i] = decode_f16(src[i]);
-    } else if (dtype == ORACLE_BF16) {
-        for (int64_t i = 0; i < n; ++i) dst[i] = decode_bf16(src[i]);
-    } else {
-        return -1;
-    }
+    if (!valid_dtype(dtype)) return -1;
+    for (int64_t i = 0; i < n; ++i) dst[i] = decode_one(src[i], dtype);
     return 0;
 }
 
@@ -178,7 +231,7 @@ int oracle_gemm_relu(const uint16_t *A, const uint16_t *B, double *C,
                      int in_dtype, int trans_b, int relu, int nthreads)
 {
     if (M < 0 || N < 0 || K < 0) return -1;
-    if (in_dtype != ORACLE_F16 && in_dtype != ORACLE_BF16) return -1;
+    if (!valid_dtype(in_dtype)) return -1;
     if (M == 0 || N == 0) return 0;
     if (!C || (K > 0 && (!A || !B))) return -1;
     set_threads(nthreads);
@@ -210,7 +263,7 @@ int oracle_gemm_relu_sampled(const uint16_t *A, const uint16_t *B,
                              int in_dtype, int trans_b, int relu, int nthreads)
 {
     if (M < 0 || N < 0 || K < 0 || count < 0) return -1;
-    if (in_dtype != ORACLE_F16 && in_dtype != ORACLE_BF16) return -1;
+    if (!valid_dtype(in_dtype)) return -1;
     if (count == 0) return 0;
     if (!rows || !cols || !out || (K > 0 && (!A || !B))) return -1;
     for (int64_t t = 0; t < count; ++t)
@@ -224,8 +277,8 @@ int oracle_gemm_relu_sampled(const uint16_t *A, const uint16_t *B,
         for (int64_t k = 0; k < K; ++k) {
             uint16_t av = A[i * K + k];
             uint16_t bv = trans_b ? B[j * K + k] : B[k * N + j];
-            double a = in_dtype == ORACLE_F16 ? decode_f16(av) : decode_bf16(av);
-            double b = in_dtype == ORACLE_F16 ? decode_f16(bv) : decode_bf16(bv);
+            double a = decode_one(av, in_dtype);
+            double b = decode_one(bv, in_dtype);
             s = s + a * b;
         }
         out[t] = apply_relu(s, relu);
@@ -242,7 +295,7 @@ int oracle_gemm_relu_rows(const uint16_t *A, const uint16_t *B,
                           int in_dtype, int trans_b, int relu, int nthreads)
 {
     if (M < 0 || N < 0 || K < 0 || nrows < 0) return -1;
-    if (in_dtype != ORACLE_F16 && in_dtype != ORACLE_BF16) return -1;
+    if (!valid_dtype(in_dtype)) return -1;
     if (nrows == 0 || N == 0) return 0;
     if (!rows || !out || (K > 0 && (!A || !B))) return -1;
     for (int64_t r = 0; r < nrows; ++r)

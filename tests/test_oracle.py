@@ -19,6 +19,7 @@ from tests.parity_util import read_golden
 from tiled_tensor_core_04_b200 import workloads as wl
 
 DTYPES = [torch.float16, torch.bfloat16]
+FP8 = [torch.float8_e4m3fn, torch.float8_e5m2]
 
 
 # --------------------------------------------------------------------------
@@ -43,6 +44,31 @@ def test_decode_bf16_every_pattern(oracle_mod):
     nan = np.isnan(want)
     assert np.array_equal(np.isnan(got), nan)
     assert np.array_equal(got[~nan], want[~nan])
+
+
+@pytest.mark.parametrize("dtype", FP8)
+def test_decode_fp8_every_pattern(oracle_mod, dtype):
+    # the 8-bit formats against torch's own conversion, all 256 patterns
+    bits = np.arange(256, dtype=np.uint16)
+    got = oracle_mod.decode(bits, dtype)
+    want = torch.from_numpy(bits.astype(np.uint8)).view(dtype).double().numpy()
+    nan = np.isnan(want)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], want[~nan])
+
+
+def test_decode_fp8_closed_forms(oracle_mod):
+    # OFP8 format facts: E4M3 has no infinities, max 448, NaN only at S.1111.111,
+    # min subnormal 2^-9, min normal 2^-6; E5M2 is IEEE-like, max 57344,
+    # infinity at exponent 31, min subnormal 2^-16
+    e4 = oracle_mod.decode(np.array([0x7E, 0x7F, 0x78, 0x01, 0x08, 0x38, 0xB8], np.uint16),
+                           torch.float8_e4m3fn)
+    assert e4[0] == 448.0 and np.isnan(e4[1]) and e4[2] == 256.0
+    assert e4[3] == 2.0 ** -9 and e4[4] == 2.0 ** -6 and e4[5] == 1.0 and e4[6] == -1.0
+    e5 = oracle_mod.decode(np.array([0x7B, 0x7C, 0x7D, 0x01, 0x04, 0x3C], np.uint16),
+                           torch.float8_e5m2)
+    assert e5[0] == 57344.0 and e5[1] == np.inf and np.isnan(e5[2])
+    assert e5[3] == 2.0 ** -16 and e5[4] == 2.0 ** -14 and e5[5] == 1.0
 
 
 # --------------------------------------------------------------------------
@@ -188,6 +214,36 @@ def test_brute_force_rationals(oracle_mod, dtype, trans_b, M, N, K):
             assert rel[i, j] == (ref[i, j] if ref[i, j] > 0 else 0.0)
 
 
+@pytest.mark.parametrize("dtype", FP8)
+@pytest.mark.parametrize("trans_b", [False, True])
+def test_fp8_closed_forms_and_exact_sums(oracle_mod, dtype, trans_b):
+    # ones -> exactly K; B = identity -> relu(A); small integers (exact in both
+    # formats) -> the int64 product; tiny uniform shapes -> the Fraction sum
+    M, N, K = 5, 7, 300
+    A = torch.ones(M, K, dtype=dtype)
+    B = torch.ones((N, K) if trans_b else (K, N), dtype=dtype)
+    assert np.all(oracle_mod.gemm_relu(A, B, trans_b=trans_b) == float(K))
+    A, _ = wl.make_inputs(6, 16, 16, dtype, False, "uniform", seed=2)
+    eye = torch.eye(16).to(dtype)
+    assert np.array_equal(oracle_mod.gemm_relu(A, eye, trans_b=trans_b, relu=True),
+                          A.double().clamp_min(0).numpy())
+    A, B = wl.small_int_inputs(9, 11, 37, dtype, trans_b, seed=5)
+    a, b = A.to(torch.int64).numpy(), B.to(torch.int64).numpy()
+    exact = a @ (b.T if trans_b else b)
+    assert np.array_equal(oracle_mod.gemm_relu(A, B, trans_b=trans_b, relu=False),
+                          exact.astype(np.float64))
+    A, B = wl.make_inputs(3, 4, 9, dtype, trans_b, "uniform", seed=9)
+    av = [[Fraction(float(v)) for v in row] for row in A.double().tolist()]
+    bv = [[Fraction(float(v)) for v in row] for row in B.double().tolist()]
+    ref = oracle_mod.gemm_relu(A, B, trans_b=trans_b, relu=False)
+    for i in range(3):
+        for j in range(4):
+            terms = [av[i][k] * (bv[j][k] if trans_b else bv[k][j]) for k in range(9)]
+            exact = sum(terms, Fraction(0))
+            assert abs(Fraction(ref[i, j]) - exact) <= Fraction(8 * 2.0 ** -53 * float(
+                sum(abs(t) for t in terms)))
+
+
 def test_golden_worked_example(oracle_mod):
     g = read_golden("worked_example.txt")
     for dtype in DTYPES:
@@ -286,6 +342,13 @@ def _pins_pass(o) -> bool:
         ok = np.isnan(bf)
         if not (np.array_equal(np.isnan(got), ok) and np.array_equal(got[~ok], bf[~ok])):
             return False
+        b8 = np.arange(256, dtype=np.uint16)
+        for dtype in FP8:
+            want = torch.from_numpy(b8.astype(np.uint8)).view(dtype).double().numpy()
+            got = o.decode(b8, dtype)
+            ok = np.isnan(want)
+            if not (np.array_equal(np.isnan(got), ok) and np.array_equal(got[~ok], want[~ok])):
+                return False
         for dtype in DTYPES:
             for tb in (False, True):
                 M, N, K = 9, 11, 37
@@ -323,6 +386,10 @@ MUTANTS = [
      "    if (trans_b) {\n        for (int64_t j = j0"),
     ("fp16 exponent bias off by one", "expo - 25);", "expo - 24);"),
     ("bf16 implicit bit dropped", "(frac | 0x80)", "(frac)"),
+    ("e4m3 exponent bias off by one", "expo - 10);", "expo - 11);"),
+    ("e4m3 read as IEEE (exponent 15 all infinity/NaN)", "if (expo == 0xf && frac == 0x7)",
+     "if (expo == 0xf)"),
+    ("e5m2 subnormal scale wrong", "ldexp((double)frac, -16);", "ldexp((double)frac, -15);"),
     ("sampled path reads B with the other layout",
      "trans_b ? B[j * K + k] : B[k * N + j]", "trans_b ? B[k * N + j] : B[j * K + k]"),
 ]
