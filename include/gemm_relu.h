@@ -61,8 +61,22 @@ extern "C" {
 typedef enum {
     GEMM_F16 = 0,  /* IEEE binary16 */
     GEMM_BF16 = 1, /* bfloat16 */
-    GEMM_F32 = 2   /* IEEE binary32 (output only) */
+    GEMM_F32 = 2,  /* IEEE binary32 (output only) */
+    GEMM_E4M3 = 3, /* 8-bit floating point E4M3, OCP OFP8 "fn" (input only) */
+    GEMM_E5M2 = 4  /* 8-bit floating point E5M2, OCP OFP8 (input only) */
 } gemm_dtype_t;
+/* 8-bit inputs (E4M3 / E5M2; A and B of the same type), products summed in
+ * fp32 on the tensor cores (tcgen05 kind::f8f6f4) like the 16-bit types:
+ *   - B must be stored N x K (trans_b = 1): 8-bit operands are read K-major;
+ *     trans_b = 0 returns GEMM_ERR_UNSUPPORTED_DTYPE;
+ *   - rows are not re-pitched: K must be a multiple of 16 and A, B 16-byte
+ *     aligned, else GEMM_ERR_MISALIGNED;
+ *   - the CTA-pair kernel with 256 x 512 or 256 x 448 tiles is the only 8-bit
+ *     path: cta_pair, split_k, swap_ab, stream_k and stage_k are ignored, and
+ *     wide = 2 counts as auto;
+ *   - gemm_relu_splitk_noalloc does not take them.
+ * This extends the method of the TileLang notes (16-bit inputs) to the 8-bit
+ * tensor-core formats of sm_100a; the pages give no 8-bit example. */
 
 typedef enum {
     GEMM_OK = 0,

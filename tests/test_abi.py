@@ -280,3 +280,27 @@ def test_autotune_candidates_cover_the_tile_shapes(lib):
     sk = [o for o in at.candidates(64, 8192, 8192, 0, 0, False) if o and o.get("swap_ab")]
     assert {o.get("split_k") for o in sk if "split_k" in o} >= {1, 4, 8}
     assert any(o.get("stream_k") for o in sk)
+
+
+# ---------------------------------------------------------------- 8-bit inputs (planner)
+def test_fp8_plans(lib):
+    E4, E5 = g.GEMM_E4M3, g.GEMM_E5M2
+    p = g.gemm_relu_plan(8192, 8192, 8192, E4, g.GEMM_F16, True)
+    assert (p["cta_pair"], p["tile_n"], p["tile_k"], p["kblocks"], p["split_k"]) == (1, 512, 128, 64, 1)
+    p = g.gemm_relu_plan(8192, 7168, 8192, E5, g.GEMM_F32, True)
+    assert p["tile_n"] == 448 and p["kblocks"] == 64
+    # knobs that select another kernel are ignored: the wide pair is the 8-bit path
+    p = g.gemm_relu_plan(64, 4096, 4096, E4, g.GEMM_F16, True,
+                         options={"split_k": 4, "cta_pair": g.GEMM_CTA_SINGLE, "swap_ab": 1,
+                                  "wide": 2})
+    assert (p["cta_pair"], p["swap_ab"], p["split_k"]) == (1, 0, 1) and p["tile_n"] in (448, 512)
+    assert g.gemm_relu_plan(512, 1000, 256, E4, g.GEMM_F16, True, options={"wide": 3})["tile_n"] == 448
+    with pytest.raises(g.GemmError) as e:                      # B must be K-major
+        g.gemm_relu_plan(512, 512, 512, E4, g.GEMM_F16, False)
+    assert e.value.status == g.GEMM_ERR_UNSUPPORTED_DTYPE
+    with pytest.raises(g.GemmError) as e:                      # 8-bit rows are not re-pitched
+        g.gemm_relu_plan(512, 512, 520, E4, g.GEMM_F16, True)
+    assert e.value.status == g.GEMM_ERR_MISALIGNED
+    with pytest.raises(g.GemmError) as e:                      # no 8-bit output
+        g.gemm_relu_plan(512, 512, 512, E4, E4, True)
+    assert e.value.status == g.GEMM_ERR_UNSUPPORTED_DTYPE

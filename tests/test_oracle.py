@@ -321,7 +321,10 @@ def test_workload_table():
     bt = wl.WORKLOADS["bt8192x7168x8192_bf16_f32"]
     assert bt.trans_b and bt.out_dtype == torch.float32 and bt.in_dtype == torch.bfloat16
     assert bt.N == 32 * 224 and bt.M == 32 * 256
-    assert [w.seed for w in wl.WORKLOADS.values()] == [0, 1, 2, 3, 4, 4, 4]
+    assert [w.seed for w in wl.WORKLOADS.values()] == [0, 1, 2, 3, 4, 4, 4, 5]
+    f8 = wl.WORKLOADS["fp8e4m3_8192_bt_f16"]
+    assert f8.in_dtype == torch.float8_e4m3fn and f8.trans_b and f8.algorithmic_bytes == (
+        2 * 8192 * 8192 + 2 * 8192 * 8192)
 
 
 # --------------------------------------------------------------------------

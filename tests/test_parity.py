@@ -199,7 +199,7 @@ def sampled_check(w: wl.Workload, C: torch.Tensor, A, B):
 
 
 @pytest.mark.parametrize("name", ["square4096_f16", "square8192_f16",
-                                  "bt8192x7168x8192_bf16_f32"])
+                                  "bt8192x7168x8192_bf16_f32", "fp8e4m3_8192_bt_f16"])
 def test_full_size_workloads_sampled(name):
     w = wl.WORKLOADS[name]
     A, B = wl.workload_inputs(w)
@@ -219,6 +219,46 @@ def test_full_size_workloads_other_tile(name, opt):
     C = run(A, B, w.out_dtype, w.trans_b, True, VARIANTS[opt])
     assert torch.isfinite(C.float()).all() and (C.float() >= 0).all()
     sampled_check(w, C, A, B)
+
+
+# ---------------------------------------------------------------- 8-bit inputs
+F8 = [torch.float8_e4m3fn, torch.float8_e5m2]
+
+
+@pytest.mark.parametrize("in_dtype", F8)
+@pytest.mark.parametrize("out_dtype", [F16, BF16, F32])
+@pytest.mark.parametrize("variant", ["auto", "wide", "wide448", "wide448_few"])
+@pytest.mark.parametrize("M,N,K", [(1, 1, 16), (256, 512, 128), (257, 449, 144),
+                                   (300, 520, 320), (520, 1400, 1024)])
+def test_fp8_against_the_oracle(in_dtype, out_dtype, variant, M, N, K):
+    # K multiples of 16 (8-bit rows must be 16-byte aligned); B stored (N, K)
+    full_case(M, N, K, in_dtype, out_dtype, True, True, VARIANTS[variant], seed=M + K)
+
+
+@pytest.mark.parametrize("in_dtype", F8)
+@pytest.mark.parametrize("relu", [False, True])
+def test_fp8_closed_forms(in_dtype, relu):
+    A = torch.ones(300, 1024, dtype=in_dtype)
+    B = torch.ones(520, 1024, dtype=in_dtype)
+    assert (run(A, B, F16, True, relu).float() == 1024).all()       # exactly K
+    A, _ = wl.make_inputs(333, 256, 256, in_dtype, False, "uniform", seed=5)
+    C = run(A, torch.eye(256).to(in_dtype), F32, True, relu)          # B = I: relu(A) exactly
+    want = A.float().clamp_min(0) if relu else A.float()
+    assert torch.equal(C, want)
+    A, B = wl.small_int_inputs(300, 520, 1024, in_dtype, True, seed=6)
+    exact = A.to(torch.int64) @ B.to(torch.int64).t()
+    C = run(A, B, F32, True, relu)
+    assert torch.equal(C.to(torch.int64), exact.clamp_min(0) if relu else exact)
+
+
+def test_fp8_refusals_launch_nothing():
+    A = torch.ones(64, 64, dtype=torch.float8_e4m3fn, device="cuda")
+    C = torch.full((64, 64), 7.0, dtype=F16, device="cuda")
+    for tb, K in ((False, 64), (True, 40)):       # B not K-major; K not a multiple of 16
+        st = g.gemm_relu(A, A, C, 64, 64, K, torch.float8_e4m3fn, F16, tb, True, check=False)
+        assert st in (g.GEMM_ERR_UNSUPPORTED_DTYPE, g.GEMM_ERR_MISALIGNED)
+    torch.cuda.synchronize()
+    assert (C.float() == 7).all()
 
 
 # ---------------------------------------------------------------- closed forms

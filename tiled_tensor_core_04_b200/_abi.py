@@ -15,7 +15,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libgemmrelu.so")
 
-GEMM_F16, GEMM_BF16, GEMM_F32 = 0, 1, 2
+GEMM_F16, GEMM_BF16, GEMM_F32, GEMM_E4M3, GEMM_E5M2 = 0, 1, 2, 3, 4
 GEMM_CTA_AUTO, GEMM_CTA_PAIR, GEMM_CTA_SINGLE = 0, 1, 2
 
 STATUS = {
@@ -41,7 +41,8 @@ EXPORTS = (
 # size of the static device array behind gemm_relu_splitk_noalloc (header constant)
 NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
-_DTYPE_CODE = {torch.float16: GEMM_F16, torch.bfloat16: GEMM_BF16, torch.float32: GEMM_F32}
+_DTYPE_CODE = {torch.float16: GEMM_F16, torch.bfloat16: GEMM_BF16, torch.float32: GEMM_F32,
+               torch.float8_e4m3fn: GEMM_E4M3, torch.float8_e5m2: GEMM_E5M2}
 
 
 class GemmOptions(ctypes.Structure):

@@ -84,19 +84,21 @@ int variant_index(bool pair, int kk, bool b_mn, gemm_dtype_t out)
 using WideKernelFn = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap,
                               const GemmParams);
 
-template <bool BMN, int BNH>
+template <bool BMN, int BNH, bool F8 = false>
 WideKernelFn pick_wide_out(gemm_dtype_t out)
 {
     switch (out) {
-    case GEMM_F16: return gemm_relu_wide_kernel<BMN, __half, BNH>;
-    case GEMM_BF16: return gemm_relu_wide_kernel<BMN, __nv_bfloat16, BNH>;
-    default: return gemm_relu_wide_kernel<BMN, float, BNH>;
+    case GEMM_F16: return gemm_relu_wide_kernel<BMN, __half, BNH, F8>;
+    case GEMM_BF16: return gemm_relu_wide_kernel<BMN, __nv_bfloat16, BNH, F8>;
+    default: return gemm_relu_wide_kernel<BMN, float, BNH, F8>;
     }
 }
 
-// bnh: MMA half width (tile_n / 2), 256 or 224 (224 with b_mn == false only)
-WideKernelFn pick_wide(bool b_mn, int bnh, gemm_dtype_t out)
+// bnh: MMA half width (tile_n / 2), 256 or 224 (224 with b_mn == false only);
+// f8: 8-bit operands (b_mn == false only)
+WideKernelFn pick_wide(bool b_mn, int bnh, gemm_dtype_t out, bool f8 = false)
 {
+    if (f8) return bnh == 224 ? pick_wide_out<false, 224, true>(out) : pick_wide_out<false, 256, true>(out);
     if (bnh == 224) return pick_wide_out<false, 224>(out);
     return b_mn ? pick_wide_out<true, 256>(out) : pick_wide_out<false, 256>(out);
 }
@@ -166,7 +168,7 @@ struct DeviceInfo {
     int max_pair_clusters = 0;
     bool attr_set[18] = {};
     bool skinny_attr_set[24] = {};
-    bool wide_attr_set[9] = {};
+    bool wide_attr_set[15] = {};
 };
 
 std::mutex g_dev_mutex;
@@ -196,11 +198,11 @@ gemm_status_t ensure_skinny_attr(DeviceInfo &d, int np, bool b_mn, gemm_dtype_t 
     return GEMM_OK;
 }
 
-gemm_status_t ensure_wide_attr(DeviceInfo &d, bool b_mn, int bnh, gemm_dtype_t out)
+gemm_status_t ensure_wide_attr(DeviceInfo &d, bool b_mn, int bnh, gemm_dtype_t out, bool f8)
 {
-    const int v = (bnh == 224 ? 6 : b_mn ? 3 : 0) + static_cast<int>(out);
+    const int v = (f8 ? (bnh == 224 ? 12 : 9) : bnh == 224 ? 6 : b_mn ? 3 : 0) + static_cast<int>(out);
     if (d.wide_attr_set[v]) return GEMM_OK;
-    cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void *>(pick_wide(b_mn, bnh, out)),
+    cudaError_t e = cudaFuncSetAttribute(reinterpret_cast<const void *>(pick_wide(b_mn, bnh, out, f8)),
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, wide_smem(bnh));
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(wide)");
     d.wide_attr_set[v] = true;
@@ -259,7 +261,8 @@ gemm_status_t device_info(DeviceInfo **out)
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
 
-size_t dtype_size(gemm_dtype_t t) { return t == GEMM_F32 ? 4 : 2; }
+bool is_f8(gemm_dtype_t t) { return t == GEMM_E4M3 || t == GEMM_E5M2; }
+size_t dtype_size(gemm_dtype_t t) { return t == GEMM_F32 ? 4 : is_f8(t) ? 1 : 2; }
 
 struct Layout {
     // byte offsets inside the workspace
@@ -275,17 +278,30 @@ gemm_status_t make_plan(int64_t M, int64_t N, int64_t K, gemm_dtype_t in, gemm_d
                         gemm_relu_plan_t *plan, Layout *lay)
 {
     if (M < 0 || N < 0 || K < 0 || num_sms <= 0) return GEMM_ERR_INVALID_ARG;
-    if (in != GEMM_F16 && in != GEMM_BF16) return GEMM_ERR_UNSUPPORTED_DTYPE;
+    if (in != GEMM_F16 && in != GEMM_BF16 && !is_f8(in)) return GEMM_ERR_UNSUPPORTED_DTYPE;
+    // 8-bit operands are read K-major only (B stored N x K)
+    if (is_f8(in) && !trans_b) return GEMM_ERR_UNSUPPORTED_DTYPE;
     if (out != GEMM_F16 && out != GEMM_BF16 && out != GEMM_F32) return GEMM_ERR_UNSUPPORTED_DTYPE;
     // the kernels index rows/columns with 32-bit ints; TMA dims must be < 2^32
     if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX - 2 * kBK) return GEMM_ERR_INVALID_ARG;
     gemm_relu_options_t o = {};
     if (opts) o = *opts;
+    const bool f8 = is_f8(in);
     if (o.cta_pair < 0 || o.cta_pair > 2 || o.split_k < 0 || o.panel < 0 || o.max_ctas < 0 ||
         (o.stage_k != 0 && o.stage_k != 64 && o.stage_k != 128) || o.l2_hint_a < 0 ||
         o.l2_hint_a > 2 || o.l2_hint_b < 0 || o.l2_hint_b > 2 || o.c_streaming < 0 || o.c_streaming > 1 || o.swap_ab < 0 || o.swap_ab > 2 ||
         o.stream_k < 0 || o.stream_k > 1 || o.wide < 0 || o.wide > 3)
         return GEMM_ERR_INVALID_ARG;
+    if (f8) {
+        // the wide CTA-pair kernel is the 8-bit path: no split-K, swap-AB,
+        // 1-CTA or 256 x 256 tiles; `wide` still picks 512 (1) or 448 (3)
+        o.cta_pair = GEMM_CTA_PAIR;
+        o.split_k = 1;
+        o.swap_ab = 2;
+        o.stream_k = 0;
+        o.stage_k = 0;
+        if (o.wide == 2) o.wide = 0;
+    }
 
     gemm_relu_plan_t p = {};
     p.tile_n = kBN;
@@ -384,7 +400,9 @@ gemm_status_t make_plan(int64_t M, int64_t N, int64_t K, gemm_dtype_t in, gemm_d
             const int64_t cost_512 = 16 * ceil_div(tiles_m * ceil_div(N, 512), clusters);
             const int64_t cost_448 = trans_b ? 14 * ceil_div(tiles_m * ceil_div(N, 448), clusters)
                                              : INT64_MAX;
-            if (cost_512 <= cost_sq && cost_512 <= cost_448)
+            if (f8)  // no 256 x 256 kernel for 8-bit operands
+                wide_n = cost_512 <= cost_448 ? 512 : 448;
+            else if (cost_512 <= cost_sq && cost_512 <= cost_448)
                 wide_n = 512;
             else if (cost_448 <= cost_sq)
                 wide_n = 448;
@@ -394,7 +412,7 @@ gemm_status_t make_plan(int64_t M, int64_t N, int64_t K, gemm_dtype_t in, gemm_d
     // the 256 x 256 pair kernel takes 128 of K per pipeline stage unless asked
     // for 64; the wide kernel takes 64
     const int kk = (pair && !wide && o.stage_k != 64) ? 2 : 1;
-    p.tile_k = kBK * kk;
+    p.tile_k = kBK * kk * (f8 ? 2 : 1);  // elements: a K block is 128 bytes of a row
     p.kblocks = static_cast<int>(ceil_div(K, p.tile_k));
     if (wide) p.tile_n = wide_n;
     const int64_t tiles_n_used = wide ? ceil_div(N, wide_n) : tiles_n;
@@ -420,10 +438,13 @@ gemm_status_t make_plan(int64_t M, int64_t N, int64_t K, gemm_dtype_t in, gemm_d
     }  // !swap
 
     // TMA reads rows whose byte pitch and base address are 16-byte aligned
-    const int64_t a_row_bytes = K * 2;
-    const int64_t b_row_bytes = (trans_b ? K : N) * 2;
+    const int64_t esz = static_cast<int64_t>(dtype_size(in));
+    const int64_t a_row_bytes = K * esz;
+    const int64_t b_row_bytes = (trans_b ? K : N) * esz;
     p.pack_a = (o.force_pack || misaligned16(A) || (a_row_bytes % 16) != 0) ? 1 : 0;
     p.pack_b = (o.force_pack || misaligned16(B) || (b_row_bytes % 16) != 0) ? 1 : 0;
+    // 8-bit rows are not re-pitched: they must already suit TMA
+    if (f8 && (p.pack_a || p.pack_b) && K > 0 && M > 0 && N > 0) return GEMM_ERR_MISALIGNED;
     if (K == 0 || M == 0 || N == 0) p.pack_a = p.pack_b = 0;
 
     Layout l;
@@ -568,11 +589,12 @@ gemm_status_t encode_2d_uncached(CUtensorMap *map, const void *base, gemm_dtype_
     }
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(pitch_elems) *
-                             static_cast<cuuint64_t>(dt == GEMM_F32 ? 4 : 2)};
+                             static_cast<cuuint64_t>(dtype_size(dt))};
     cuuint32_t box[2] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_outer)};
     cuuint32_t estr[2] = {1, 1};
     const CUtensorMapDataType type = dt == GEMM_F32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
                                      : dt == GEMM_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                     : is_f8(dt)       ? CU_TENSOR_MAP_DATA_TYPE_UINT8
                                                        : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
     CUresult r = fn(map, type, 2, const_cast<void *>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -588,9 +610,10 @@ gemm_status_t encode_2d_uncached(CUtensorMap *map, const void *base, gemm_dtype_
 // tcgen05 instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A/B type
 // (bits 7-9 / 10-12: 0 fp16, 1 bf16), A K-major (bit 15 = 0), B major (bit
 // 16: 0 K-major, 1 MN-major), N >> 3 (bits 17-22), M >> 4 (bits 24-28).
+// The same type fields name the 8-bit formats of kind::f8f6f4 (0 E4M3, 1 E5M2).
 uint32_t make_idesc(gemm_dtype_t in, bool b_mn, int mma_m, int mma_n, bool a_mn = false)
 {
-    const uint32_t t = in == GEMM_BF16 ? 1u : 0u;
+    const uint32_t t = (in == GEMM_BF16 || in == GEMM_E5M2) ? 1u : 0u;
     return (1u << 4) | (t << 7) | (t << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
            (static_cast<uint32_t>(mma_n >> 3) << 17) | (static_cast<uint32_t>(mma_m >> 4) << 24);
 }
@@ -764,13 +787,16 @@ gemm_status_t run(const void *A, const void *B, void *C, int64_t M, int64_t N, i
     const int bnh = plan.tile_n / 2;  // wide kernels: MMA half width
     // rows of a K-major B box: this CTA's share of one MMA's N
     const int bn_cta = wide ? bnh / 2 : pair ? kBN / 2 : kBN;
+    // a K block is one 128-byte row segment: 64 16-bit or 128 8-bit elements
+    const bool f8 = is_f8(in);
+    const int kbox = f8 ? 2 * kBK : kBK;
     CUtensorMap tmA, tmB;
-    st = encode_2d(&tmA, a_src, in, K, M, a_pitch, kBK, kBM);
+    st = encode_2d(&tmA, a_src, in, K, M, a_pitch, kbox, kBM);
     if (st != GEMM_OK) return st;
     if (b_mn)
         st = encode_2d(&tmB, b_src, in, N, K, b_pitch, 64, kBK);
     else
-        st = encode_2d(&tmB, b_src, in, K, N, b_pitch, kBK, bn_cta);
+        st = encode_2d(&tmB, b_src, in, K, N, b_pitch, kbox, bn_cta);
     if (st != GEMM_OK) return st;
 
     const bool split = plan.split_k > 1;
@@ -809,7 +835,8 @@ gemm_status_t run(const void *A, const void *B, void *C, int64_t M, int64_t N, i
     }
     {
         std::lock_guard<std::mutex> lock(g_dev_mutex);
-        st = wide ? ensure_wide_attr(*dev, b_mn, bnh, kout) : ensure_kernel_attr(*dev, pair, kk, b_mn, kout);
+        st = wide ? ensure_wide_attr(*dev, b_mn, bnh, kout, f8)
+                  : ensure_kernel_attr(*dev, pair, kk, b_mn, kout);
     }
     if (st != GEMM_OK) return st;
 
@@ -825,7 +852,7 @@ gemm_status_t run(const void *A, const void *B, void *C, int64_t M, int64_t N, i
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pair ? 1 : 0;
-    cudaError_t e = wide ? cudaLaunchKernelEx(&cfg, pick_wide(b_mn, bnh, kout), tmA, tmB, tmC, p)
+    cudaError_t e = wide ? cudaLaunchKernelEx(&cfg, pick_wide(b_mn, bnh, kout, f8), tmA, tmB, tmC, p)
                          : cudaLaunchKernelEx(&cfg, pick_kernel(pair, kk, b_mn, kout), tmA, tmB, p);
     if (e != cudaSuccess) return cuda_fail(e, "gemm kernel launch");
 
@@ -1033,6 +1060,7 @@ extern "C" gemm_status_t gemm_relu_splitk_noalloc(const void *A, const void *B, 
 {
     cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
     if (split_k < 0) return GEMM_ERR_INVALID_ARG;
+    if (is_f8(in)) return GEMM_ERR_UNSUPPORTED_DTYPE;  // no 8-bit split-K kernel
     gemm_relu_options_t o = {};
     o.cta_pair = GEMM_CTA_SINGLE;
     o.split_k = split_k;

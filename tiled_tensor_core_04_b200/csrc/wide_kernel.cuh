@@ -146,7 +146,11 @@ __device__ __forceinline__ void store_chunk(OutT *dst, const uint32_t (&v)[32], 
 // 10 warps: three share one SM sub-partition's 16 K registers, so at most
 // 168 registers per thread; the epilogue holds 128 accumulator columns per
 // thread at once.
-template <bool B_MN, typename OutT, int BNH>
+// F8: 8-bit operands (E4M3 / E5M2, kind::f8f6f4).  A K block is still one
+// 128-byte row segment per operand row, i.e. 128 elements instead of 64, and
+// the four K steps per block are 32 elements (32 bytes) each, so the shared
+// memory layout, descriptors and byte counts are those of the 16-bit case.
+template <bool B_MN, typename OutT, int BNH, bool F8 = false>
 __global__ void __launch_bounds__(kWideThreads, 1)
     gemm_relu_wide_kernel(const __grid_constant__ CUtensorMap tmA,
                           const __grid_constant__ CUtensorMap tmB,
@@ -154,6 +158,8 @@ __global__ void __launch_bounds__(kWideThreads, 1)
 {
     using Cfg = WideCfg<BNH>;
     static_assert(!B_MN || BNH == 256, "MN-major B needs 256-column halves");
+    static_assert(!F8 || !B_MN, "8-bit operands are read K-major");
+    constexpr int kKE = F8 ? 2 * kBK : kBK;  // K elements per block
     constexpr int kStages = Cfg::kStages;
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -227,7 +233,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                     const uint32_t fb_leader = map_shared_to_rank(fb, 0);
                     const uint32_t a_dst = tiles_base + static_cast<uint32_t>(stage * Cfg::kStageBytes);
                     const uint32_t b_dst = a_dst + Cfg::kABytes;
-                    const int kx = kb * kBK;
+                    const int kx = kb * kKE;
                     if (rank == 0) mbar_arrive_expect_tx(fb, Cfg::kTxBytes);
                     tma_load_2d_pair_hint(a_dst, &tmA, fb_leader, kx, m_row, pol_a);
 #pragma unroll
@@ -272,17 +278,22 @@ __global__ void __launch_bounds__(kWideThreads, 1)
             constexpr uint64_t kStageStep = Cfg::kStageBytes >> 4;
             constexpr uint64_t kHalfStep = Cfg::kBHalf >> 4;
             const uint32_t idesc = p.idesc;
-            // four K = 16 MMAs of one stage into accumulator half h
+            // four MMAs (K = 16 elements, or 32 for 8-bit operands: 32 bytes
+            // each) of one stage into accumulator half h
             auto issue_half = [&](int s, int h, bool first) {
                 const uint64_t so = static_cast<uint64_t>(s) * kStageStep;
                 // half h accumulates at TMEM column 256 * h (for BNH = 224 too)
                 const uint32_t d = tmem_base + static_cast<uint32_t>(h * kBN);
 #pragma unroll
-                for (int k = 0; k < kBK / 16; ++k)
-                    umma_f16<2>(d, a_desc0 + so + static_cast<uint64_t>(k) * kAStep,
-                                b_desc0 + so + static_cast<uint64_t>(h) * kHalfStep +
-                                    static_cast<uint64_t>(k) * kBStep,
-                                idesc, (first && k == 0) ? 0u : 1u);
+                for (int k = 0; k < kBK / 16; ++k) {
+                    const uint64_t ad = a_desc0 + so + static_cast<uint64_t>(k) * kAStep;
+                    const uint64_t bd = b_desc0 + so + static_cast<uint64_t>(h) * kHalfStep +
+                                        static_cast<uint64_t>(k) * kBStep;
+                    if constexpr (F8)
+                        umma_f8<2>(d, ad, bd, idesc, (first && k == 0) ? 0u : 1u);
+                    else
+                        umma_f16<2>(d, ad, bd, idesc, (first && k == 0) ? 0u : 1u);
+                }
             };
             auto advance = [&](int &s, uint32_t &ph) {
                 if (++s == kStages) {

@@ -54,6 +54,7 @@ class Workload:
 
 
 F16, BF16, F32 = torch.float16, torch.bfloat16, torch.float32
+E4M3 = torch.float8_e4m3fn
 
 WORKLOADS = {
     w.name: w
@@ -71,6 +72,10 @@ WORKLOADS = {
                  note="skinny M: memory-bound on B, split-K"),
         Workload("skinny16x16384x4096_f16", 16, 16384, 4096, F16, F16, False, "uniform", 4,
                  note="skinny M: memory-bound on B, split-K"),
+        Workload("fp8e4m3_8192_bt_f16", 8192, 8192, 8192, E4M3, F16, True, "uniform", 5,
+                 note="8-bit (E4M3) inputs on the kind::f8f6f4 tensor cores, B stored (N, K), "
+                      "fp16 out: the FP8 follow-on of the same method, not a configuration "
+                      "of the essay"),
     ]
 }
 
