@@ -49,9 +49,10 @@ L2_BYTES = 126 * 2 ** 20
 # on (a changed kernel reports null until it is profiled again).
 NCU_TRAFFIC_BYTES: dict[str, dict[str, float]] = {
     # profiles/gemm_relu_wide_kernel_*.md, profiles/gemm_relu_skinny_kernel_*.md
-    "52b67171c34c9af6": {"square8192_f16": 743.915264e6 + 120.3392e6,
-                         "bt8192x7168x8192_bf16_f32": 692.724736e6 + 207.65312e6,
-                         "skinny64x8192x8192_f16": 135.314432e6 + 3.935488e6},
+    "448ad32fb0119d85": {"square8192_f16": 755.22304e6 + 120.565504e6,
+                         "fp8e4m3_8192_bt_f16": 318.143232e6 + 116.811776e6,
+                         "bt8192x7168x8192_bf16_f32": 691.881472e6 + 208.086784e6,
+                         "skinny64x8192x8192_f16": 135.312896e6 + 4.084992e6},
 }
 
 _DT = {torch.float16: "f16", torch.bfloat16: "bf16", torch.float32: "f32",
