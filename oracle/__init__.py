@@ -14,7 +14,7 @@ TileLang" essay, section 2):
 with op(B) = B for B stored (K, N) and op(B) = B^T for B stored (N, K)
 (``trans_b``).  The result is returned unrounded as float64.  ``round_output``
 gives the oracle's own image in the output dtype, for reporting only; parity
-is judged against the unrounded value.
+is compared against the unrounded value.
 """
 from __future__ import annotations
 
